@@ -1,0 +1,354 @@
+"""Benchmark: gated SwiGLU FFN decode, Llama-7B shape (d 4096, ffn 11008, bf16), batch 1.
+
+One step = one pass of the whole hot path over L distinct layers (each with its own
+packed weight copy and its own resident input): per layer the three gates
+(top-K of |x*c|), the three sparse products and the SwiGLU glue, i.e. one
+sparse_ffn_swiglu call. The L weight copies (2.2 GB at L = 8) exceed the 126 MB L2,
+so every step streams its kept rows from HBM.
+
+Printed (rank 0, one JSON line): effective HBM GB/s on the bytes the kept rows and the
+vectors require (value; whole job), us per layer, the roofline of the fused kernel
+against the measured HBM copy bandwidth, the dense comparator (the same kernel with
+every channel kept), the end-to-end figure through the C ABI with host buffers, and
+the CPU oracle's time on a bounded sample.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--p 0.5] [--layers 8]
+  python bench.py --impl reference ...   # the CPU oracle, timed on the host cores
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "µs/layer & effective HBM GB/s (% of peak), Llama-7B FFN sparse GEMV, bs1"
+D, FFN = 4096, 11008
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def layer_bytes(kg: int, ku: int, kd: int, d: int = D, ffn: int = FFN) -> int:
+    """Algorithmic HBM bytes of one layer: the kept rows of the three bf16 weights plus
+    the vectors that must cross HBM (x bf16, c_gate/c_up/c_down float32, y float32)."""
+    rows = (kg + ku) * ffn * 2 + kd * d * 2
+    vecs = d * 2 + 2 * d * 4 + ffn * 4 + d * 4
+    return rows + vecs
+
+
+# ------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------
+
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------
+# the CPU oracle leg (reference arm and cpu_baseline)
+# ------------------------------------------------------------------------------------
+
+
+def oracle_sample(p: float, budget_s: float = 12.0, max_tokens: int = 20) -> dict:
+    """Time the CPU oracle's per-token FFN (select + float64 products) on one layer of
+    the same workload, as many tokens as fit in about budget_s seconds."""
+    import oracle as O
+
+    try:
+        from threadpoolctl import threadpool_info
+        blas_threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        blas_threads = 1
+    cfg = synth.make_llama7b_ffn(batch=max_tokens, p=p)
+    Wg, Wu, Wd = (O.widen_bf16(cfg[k]) for k in ("Wg", "Wu", "Wd"))
+    cg, cu, cd = O.col_norms(Wg), O.col_norms(Wu), O.col_norms(Wd)
+    x32 = synth.f32_from_bf16_bits(cfg["x"])
+    times = []
+    t_all = time.perf_counter()
+    for b in range(max_tokens):
+        t0 = time.perf_counter()
+        O.ffn_swiglu(Wg, Wu, Wd, cg, cu, cd, x32[b], cfg["k_gate"], cfg["k_up"], cfg["k_down"])
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all > budget_s and len(times) >= 3:
+            break
+    us = statistics.median(times) * 1e6
+    nbytes = layer_bytes(cfg["k_gate"], cfg["k_up"], cfg["k_down"])
+    return {"us_per_layer": us, "gbs": nbytes / (us * 1e-6) / 1e9, "tokens": len(times),
+            "cores": int(blas_threads), "host_cpus": os.cpu_count()}
+
+
+# ------------------------------------------------------------------------------------
+# the GPU arm
+# ------------------------------------------------------------------------------------
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--p", type=float, default=0.5, help="dropped fraction per projection")
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    kg = synth.keep_count(args.p, D)
+    kd = synth.keep_count(args.p, FFN)
+    nbytes = layer_bytes(kg, kg, kd)
+    config = {"workload": f"llama7b_ffn_4096x11008_bf16 decode bs1, top-K per projection at "
+                          f"{int(round(args.p * 100))}% sparsity (K={kg}/{kg}/{kd})",
+              "d": D, "ffn": FFN, "batch": 1, "p": args.p, "layers_per_step": args.layers,
+              "l2": "inputs larger than L2: distinct weight copies per layer", "parallelism": f"replicas{world}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        r = oracle_sample(args.p)
+        us = r["us_per_layer"]
+        line = {"metric": METRIC, "impl": "reference", "value": r["gbs"], "unit": "GB/s", "us_per_layer": us,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": us * args.layers / 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": r["gbs"], "unit": "GB/s", "cores": r["cores"], "kind": "oracle",
+                                 "sample": f"{r['tokens']} tokens of one layer (median per token)"},
+                "e2e": {"value": r["gbs"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import free_activation_sparse_b200 as W
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- untimed setup: L layers of weights (packed + norms on the GPU), inputs ----
+    L = args.layers
+    layers, xs = [], []
+    for l in range(L):
+        cfg = synth.make_llama7b_ffn(batch=1, p=args.p, layer=l + 1000 * rank)
+        up = [torch.from_numpy(cfg[k].view(np.int16)).cuda().view(torch.bfloat16) for k in ("Wg", "Wu", "Wd")]
+        layers.append(W.ffn_prepare(*up))
+        del up
+        xs.append(torch.from_numpy(cfg["x"].view(np.int16)).cuda().view(torch.bfloat16))
+    torch.cuda.synchronize()
+    ws = W.Workspace(W.OP_FFN_SWIGLU, D, FFN, 0, 1)
+    ys = [torch.empty((1, D), dtype=torch.float32, device="cuda") for _ in range(L)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(mode=W.GATE_TOPK, ev=None):
+        for l in range(L):
+            if ev is not None:
+                ev[l][0].record(stream)
+            W.sparse_ffn_swiglu(layers[l], xs[l], mode, kg, kg, kd, ws=ws, status=status, y=ys[l])
+            if ev is not None:
+                ev[l][1].record(stream)
+
+    def timed(mode, K, per_kernel=False):
+        evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
+               for _ in range(K)] if per_kernel else None
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for k in range(K):
+            step(mode, evs[k] if per_kernel else None)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        total_ms = t0.elapsed_time(t1)
+        kern_ms = None
+        if per_kernel:
+            kern_ms = statistics.mean(e[0].elapsed_time(e[1]) for row in evs for e in row)
+        return total_ms, kern_ms
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    total_ms, kern_ms = timed(W.GATE_TOPK, args.steps, per_kernel=True)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(total_ms)
+    kern_ms = max_over_ranks(kern_ms)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the timed region")
+
+    ms_per_step = total_ms / args.steps
+    us_layer = ms_per_step * 1e3 / L
+    gbs = world * nbytes * L * args.steps / (total_ms * 1e-3) / 1e9
+
+    # dense comparator: the same kernel with every channel kept
+    for _ in range(3):
+        step(W.GATE_DENSE)
+    dense_ms, _ = timed(W.GATE_DENSE, max(3, args.steps // 2))
+    dense_ms = max_over_ranks(dense_ms)
+    us_layer_dense = dense_ms / max(3, args.steps // 2) * 1e3 / L
+
+    # end to end through the C ABI: host x in pinned memory -> device, the call, y -> host
+    hx = [x.cpu().pin_memory() for x in xs]
+    hy = [torch.empty((1, D), dtype=torch.float32).pin_memory() for _ in range(L)]
+    dx = [torch.empty_like(x) for x in xs]
+
+    def e2e_step():
+        for l in range(L):
+            dx[l].copy_(hx[l], non_blocking=True)
+            W.sparse_ffn_swiglu(layers[l], dx[l], W.GATE_TOPK, kg, kg, kd, ws=ws, status=status, y=ys[l])
+            hy[l].copy_(ys[l], non_blocking=True)
+        torch.cuda.synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    t_e0 = torch.cuda.Event(enable_timing=True)
+    t_e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t_e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(t_e0.elapsed_time(t_e1))
+    e2e_gbs = world * nbytes * L * args.steps / (e2e_ms * 1e-3) / 1e9
+
+    peak, peak_kind = _peaks()
+    achieved = nbytes / (kern_ms * 1e-3) / 1e9
+    traffic = None
+    tf = os.path.join(ROOT, "profiles", "ffn_fused_llama7b_traffic.json")
+    if os.path.exists(tf):
+        with open(tf) as f:
+            tj = json.load(f)
+        if tj.get("p") == args.p and tj.get("kernel_sha") == _kernel_sha():
+            traffic = tj.get("dram_bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": gbs, "unit": "GB/s", "us_per_layer": us_layer,
+        "pct_of_peak": 100.0 * gbs / world / peak, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 weights, f32 accumulate", "data": "synthetic", "config": config,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
+                     "kernel": "k_ffn_fused (one launch per layer)", "bytes_per_launch": nbytes,
+                     "kernel_us": kern_ms * 1e3},
+        "dense": {"us_per_layer": us_layer_dense, "speedup": us_layer_dense / us_layer},
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "us_per_layer": e2e_ms / args.steps * 1e3 / L,
+                "h2d_bytes_per_step": L * D * 2, "d2h_bytes_per_step": L * D * 4},
+        "gpu_launches": L * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = oracle_sample(args.p)
+        line["cpu_baseline"] = {"value": r["gbs"], "unit": "GB/s", "us_per_layer": r["us_per_layer"],
+                                "cores": r["cores"], "kind": "oracle",
+                                "sample": f"{r['tokens']} tokens through one layer (median per token)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _kernel_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("common.cuh", "ffn.cu"):
+        with open(os.path.join(ROOT, "free_activation_sparse_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    main()

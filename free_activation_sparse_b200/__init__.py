@@ -1,0 +1,316 @@
+"""Weight-informed activation-sparse linear layer for LLM decode on B200 (sm_100a).
+
+A thin ctypes binding of ``libwina.so`` (the C ABI in ``include/wina.h``). Every step
+of the computation runs in the library's CUDA kernels; this module only checks tensor
+dtypes/devices, allocates outputs and workspaces through PyTorch, passes raw device
+pointers and the current CUDA stream, and turns status codes into exceptions.
+Importing it fails if the library has not been built
+(``python -m free_activation_sparse_b200.build``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+__all__ = [
+    "WinaError", "lib", "LIB_PATH", "F32", "BF16", "GATE_TOPK", "GATE_STAT", "GATE_DENSE",
+    "abi_version", "normal_quantile", "workspace_size", "Workspace", "FfnWeights",
+    "pack_in_major", "col_norms", "select_topk", "stat_topk_threshold", "sparse_matvec",
+    "sparse_ffn_swiglu", "ffn_ws_view", "ffn_prepare", "declared_symbols",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwina.so")
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "wina.h")
+
+# enums of wina.h
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_DTYPE, ERR_WORKSPACE, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT = range(7)
+F32, BF16 = 0, 1
+LAYOUT_OUT_IN, LAYOUT_IN_MAJOR = 0, 1
+GATE_TOPK, GATE_STAT, GATE_DENSE = 0, 1, 2
+OP_SELECT_TOPK, OP_STAT_THRESHOLD, OP_SPARSE_MATVEC, OP_FFN_SWIGLU = 0, 1, 2, 3
+
+
+class WinaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = int(code)
+        super().__init__(f"{where}: {lib.wina_status_string(code).decode()} (status {code})")
+
+
+class _FfnT(ctypes.Structure):
+    _fields_ = [
+        ("wt_gate", ctypes.c_void_p), ("wt_up", ctypes.c_void_p), ("wt_down", ctypes.c_void_p),
+        ("wdt", ctypes.c_int), ("c_gate", ctypes.c_void_p), ("c_up", ctypes.c_void_p),
+        ("c_down", ctypes.c_void_p), ("d", ctypes.c_int64), ("ffn", ctypes.c_int64),
+    ]
+
+
+class _FfnView(ctypes.Structure):
+    _fields_ = [("h", ctypes.c_size_t), ("idx_gate", ctypes.c_size_t), ("idx_up", ctypes.c_size_t),
+                ("idx_down", ctypes.c_size_t), ("cnt", ctypes.c_size_t)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m free_activation_sparse_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, D, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double, ctypes.c_size_t
+    E = ctypes.c_int
+    sig = {
+        "wina_abi_version": (I32, []),
+        "wina_status_string": (ctypes.c_char_p, [E]),
+        "wina_normal_quantile": (D, [D]),
+        "wina_workspace_size": (SZ, [E, I64, I64, I64, I64]),
+        "wina_ffn_ws_view": (E, [I64, I64, I64, ctypes.POINTER(_FfnView)]),
+        "wina_pack_in_major": (E, [P, E, I64, I64, P, P]),
+        "wina_col_norms": (E, [P, E, I64, I64, E, P, P]),
+        "wina_select_topk": (E, [P, E, P, I64, I64, I64, P, P, P, P]),
+        "stat_topk_threshold": (E, [P, E, I64, D, I64, P, P, P, P, I64, P, P]),
+        "sparse_matvec": (E, [P, E, I64, I64, P, P, I64, P, I64, I64, P, P, SZ, P, P]),
+        "sparse_ffn_swiglu": (E, [ctypes.POINTER(_FfnT), P, E, I64, E, I64, I64, I64, D, P, P, SZ, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+def declared_symbols() -> list[str]:
+    """Function names declared in include/wina.h (parsed from the header text)."""
+    import re
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)) - {"defined"})
+
+
+# ------------------------------------------------------------------------------------
+# marshalling helpers (no arithmetic of the method here)
+# ------------------------------------------------------------------------------------
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dt(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _cuda(t, name):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise WinaError(code, where)
+
+
+def abi_version() -> int:
+    return int(lib.wina_abi_version())
+
+
+def normal_quantile(p: float) -> float:
+    """Phi^-1(p), computed by the library's host code."""
+    return float(lib.wina_normal_quantile(float(p)))
+
+
+def workspace_size(op: int, n: int, m: int, k: int, batch: int) -> int:
+    return int(lib.wina_workspace_size(int(op), int(n), int(m), int(k), int(batch)))
+
+
+class Workspace:
+    """A zero-filled device scratch buffer for one op and size (reusable across calls
+    of that op on one stream)."""
+
+    def __init__(self, op: int, n: int, m: int, k: int, batch: int, device=None):
+        torch = _torch()
+        nbytes = max(workspace_size(op, n, m, k, batch), 256)
+        self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
+        self.nbytes = nbytes
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+# ------------------------------------------------------------------------------------
+# public calls
+# ------------------------------------------------------------------------------------
+
+
+def pack_in_major(W):
+    """W[m][n] -> Wt[n][m] (input-channel-major), same dtype."""
+    torch = _torch()
+    _cuda(W, "W")
+    m, n = W.shape
+    Wt = torch.empty((n, m), dtype=W.dtype, device=W.device)
+    _check(lib.wina_pack_in_major(_ptr(W), _dt(W), m, n, _ptr(Wt), _stream()), "wina_pack_in_major")
+    return Wt
+
+
+def col_norms(W, layout: str = "out_in"):
+    """float32 column norms c[n] of W[m][n] ('out_in') or of the packed Wt[n][m] ('in_major')."""
+    torch = _torch()
+    _cuda(W, "W")
+    if layout == "out_in":
+        m, n = W.shape
+        lay = LAYOUT_OUT_IN
+    elif layout == "in_major":
+        n, m = W.shape
+        lay = LAYOUT_IN_MAJOR
+    else:
+        raise ValueError(layout)
+    c = torch.empty(n, dtype=torch.float32, device=W.device)
+    _check(lib.wina_col_norms(_ptr(W), _dt(W), m, n, lay, _ptr(c), _stream()), "wina_col_norms")
+    return c
+
+
+def select_topk(x, c, k: int, want_scores: bool = False):
+    """Top-k gate per token: returns (idx int32 [B][k] ascending, xs float32 [B][k]
+    [, scores float32 [B][n]])."""
+    torch = _torch()
+    _cuda(x, "x")
+    _cuda(c, "c")
+    x2 = x.reshape(1, -1) if x.dim() == 1 else x
+    B, n = x2.shape
+    idx = torch.empty((B, k), dtype=torch.int32, device=x.device)
+    xs = torch.empty((B, k), dtype=torch.float32, device=x.device)
+    sc = torch.empty((B, n), dtype=torch.float32, device=x.device) if want_scores else None
+    _check(lib.wina_select_topk(_ptr(x2), _dt(x2), _ptr(c), n, k, B, _ptr(idx), _ptr(xs), _ptr(sc), _stream()),
+           "wina_select_topk")
+    return (idx, xs, sc) if want_scores else (idx, xs)
+
+
+def stat_topk_threshold(v, s: float, cap: int | None = None, status=None):
+    """Spark statistical gate per row of v: returns (idx [B][cap], xs [B][cap],
+    count [B], t [B]). Entries past count are unspecified."""
+    torch = _torch()
+    _cuda(v, "v")
+    v2 = v.reshape(1, -1) if v.dim() == 1 else v
+    B, n = v2.shape
+    cap = n if cap is None else int(cap)
+    idx = torch.empty((B, max(cap, 1)), dtype=torch.int32, device=v.device)
+    xs = torch.empty((B, max(cap, 1)), dtype=torch.float32, device=v.device)
+    count = torch.empty(B, dtype=torch.int32, device=v.device)
+    t = torch.empty(B, dtype=torch.float32, device=v.device)
+    _check(lib.stat_topk_threshold(_ptr(v2), _dt(v2), n, float(s), B, _ptr(idx), _ptr(xs), _ptr(count), _ptr(t),
+                                   cap, _ptr(status), _stream()), "stat_topk_threshold")
+    return idx[:, :cap], xs[:, :cap], count, t
+
+
+def sparse_matvec(Wt, idx, xs, k: int | None = None, count=None, ws: Workspace | None = None, status=None, y=None):
+    """y[b] = sum_r xs[b][r] * Wt[idx[b][r]] over the first k (or count[b]) entries."""
+    torch = _torch()
+    for t_, nm in ((Wt, "Wt"), (idx, "idx"), (xs, "xs"), (count, "count")):
+        _cuda(t_, nm)
+    if idx.dtype != torch.int32 or xs.dtype != torch.float32:
+        raise TypeError("idx must be int32 and xs float32")
+    idx2 = idx.reshape(1, -1) if idx.dim() == 1 else idx
+    xs2 = xs.reshape(1, -1) if xs.dim() == 1 else xs
+    n, m = Wt.shape
+    B, ld = idx2.shape
+    if k is None and count is None:
+        k = ld
+    kk = -1 if k is None else int(k)
+    if ws is None:
+        ws = Workspace(OP_SPARSE_MATVEC, n, m, ld, B, device=Wt.device)
+    if y is None:
+        y = torch.empty((B, m), dtype=torch.float32, device=Wt.device)
+    _check(lib.sparse_matvec(_ptr(Wt), _dt(Wt), n, m, _ptr(idx2), _ptr(xs2), kk, _ptr(count), ld, B, _ptr(y),
+                             ws.ptr, ws.nbytes, _ptr(status), _stream()), "sparse_matvec")
+    return y
+
+
+@dataclass
+class FfnWeights:
+    """Packed SwiGLU FFN: wt_gate/wt_up [d][ffn], wt_down [ffn][d] (input-major), and
+    the float32 column norms of W_gate, W_up (length d) and W_down (length ffn)."""
+    wt_gate: object
+    wt_up: object
+    wt_down: object
+    c_gate: object
+    c_up: object
+    c_down: object
+
+    @property
+    def d(self) -> int:
+        return int(self.wt_gate.shape[0])
+
+    @property
+    def ffn(self) -> int:
+        return int(self.wt_gate.shape[1])
+
+    def _struct(self) -> _FfnT:
+        return _FfnT(self.wt_gate.data_ptr(), self.wt_up.data_ptr(), self.wt_down.data_ptr(), _dt(self.wt_gate),
+                     self.c_gate.data_ptr(), self.c_up.data_ptr(), self.c_down.data_ptr(), self.d, self.ffn)
+
+
+def ffn_prepare(W_gate, W_up, W_down) -> FfnWeights:
+    """Offline preparation of one FFN from W_gate, W_up [ffn][d] and W_down [d][ffn]
+    (output-major, as multiplied by x): pack input-major and take column norms."""
+    return FfnWeights(pack_in_major(W_gate), pack_in_major(W_up), pack_in_major(W_down),
+                      col_norms(W_gate), col_norms(W_up), col_norms(W_down))
+
+
+def sparse_ffn_swiglu(f: FfnWeights, x, mode: int = GATE_TOPK, k_gate: int = 0, k_up: int = 0, k_down: int = 0,
+                      s: float = 0.08, ws: Workspace | None = None, status=None, y=None):
+    """Gated SwiGLU FFN for x [B][d]: returns y float32 [B][d]."""
+    torch = _torch()
+    _cuda(x, "x")
+    x2 = x.reshape(1, -1) if x.dim() == 1 else x
+    B = x2.shape[0]
+    if ws is None:
+        ws = Workspace(OP_FFN_SWIGLU, f.d, f.ffn, 0, B, device=x.device)
+    if y is None:
+        y = torch.empty((B, f.d), dtype=torch.float32, device=x.device)
+    fs = f._struct()
+    _check(lib.sparse_ffn_swiglu(ctypes.byref(fs), _ptr(x2), _dt(x2), B, int(mode), int(k_gate), int(k_up),
+                                 int(k_down), float(s), _ptr(y), ws.ptr, ws.nbytes, _ptr(status), _stream()),
+           "sparse_ffn_swiglu")
+    return y
+
+
+def ffn_ws_view(ws: Workspace, d: int, ffn: int, batch: int) -> dict:
+    """Views of the intermediate results a sparse_ffn_swiglu call leaves in `ws`:
+    h [B][ffn], idx_gate [B][d], idx_up [B][d], idx_down [B][ffn], cnt [3][B]."""
+    torch = _torch()
+    v = _FfnView()
+    _check(lib.wina_ffn_ws_view(d, ffn, batch, ctypes.byref(v)), "wina_ffn_ws_view")
+    buf = ws.buf
+
+    def take(off, count, dtype, shape):
+        nb = count * 4
+        return buf[off: off + nb].view(dtype).view(*shape)
+
+    return dict(
+        h=take(v.h, batch * ffn, torch.float32, (batch, ffn)),
+        idx_gate=take(v.idx_gate, batch * d, torch.int32, (batch, d)),
+        idx_up=take(v.idx_up, batch * d, torch.int32, (batch, d)),
+        idx_down=take(v.idx_down, batch * ffn, torch.int32, (batch, ffn)),
+        cnt=take(v.cnt, 3 * batch, torch.int32, (3, batch)),
+    )

@@ -1,0 +1,83 @@
+// Host-only entry points of the C ABI: version, status strings, the normal quantile
+// used by the Spark threshold, workspace sizes and workspace views.
+#include <math.h>
+
+#include "internal.h"
+
+namespace wina {
+
+int device_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+// Phi(z) = P(Z <= z) for a standard normal Z, via the complementary error function.
+static double normal_cdf(double z) { return 0.5 * erfc(-z / sqrt(2.0)); }
+
+}  // namespace wina
+
+using namespace wina;
+
+extern "C" int32_t wina_abi_version(void) { return WINA_ABI_VERSION; }
+
+extern "C" const char* wina_status_string(wina_status_t s) {
+  switch (s) {
+    case WINA_OK: return "ok";
+    case WINA_ERR_INVALID_ARG: return "invalid argument";
+    case WINA_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype";
+    case WINA_ERR_WORKSPACE: return "workspace too small";
+    case WINA_ERR_CAPACITY: return "more kept channels than the output capacity";
+    case WINA_ERR_CUDA: return "CUDA runtime error";
+    case WINA_ERR_TIMEOUT: return "grid barrier wait timed out";
+  }
+  return "unknown status";
+}
+
+// Standard normal quantile: solve Phi(z) = q on the lower tail (q = min(p, 1 - p), z <= 0,
+// where erfc has full relative precision) by bisection on [-40, 0] down to the spacing
+// of doubles, then two Newton steps z -= (Phi(z) - q) / phi(z); mirror for p > 1/2.
+extern "C" double wina_normal_quantile(double p) {
+  if (!(p > 0.0 && p < 1.0)) return NAN;
+  if (p == 0.5) return 0.0;
+  const double q = p < 0.5 ? p : 1.0 - p;
+  double lo = -40.0, hi = 0.0;
+  for (int it = 0; it < 200 && hi - lo > 0.0; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid <= lo || mid >= hi) break;
+    if (normal_cdf(mid) < q)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  double z = 0.5 * (lo + hi);
+  const double inv_sqrt_2pi = 0.39894228040143267794;
+  for (int it = 0; it < 2; ++it) {
+    const double pdf = inv_sqrt_2pi * exp(-0.5 * z * z);
+    if (pdf <= 0.0) break;
+    z -= (normal_cdf(z) - q) / pdf;
+  }
+  return p < 0.5 ? z : -z;
+}
+
+extern "C" size_t wina_workspace_size(wina_op_t op, int64_t n, int64_t m, int64_t k, int64_t batch) {
+  (void)k;
+  if (n < 1 || m < 1 || batch < 1) return 0;
+  switch (op) {
+    case WINA_OP_SPARSE_MATVEC: return spmv_ws_layout(m, batch).total;
+    case WINA_OP_FFN_SWIGLU: return ffn_ws_layout(n, m, batch).total;
+    default: return 0;
+  }
+}
+
+extern "C" wina_status_t wina_ffn_ws_view(int64_t d, int64_t ffn, int64_t batch, wina_ffn_ws_view_t* out) {
+  if (d < 1 || ffn < 1 || batch < 1 || !out) return WINA_ERR_INVALID_ARG;
+  const FfnWs L = ffn_ws_layout(d, ffn, batch);
+  out->h = L.h;
+  out->idx_gate = L.idx_gate;
+  out->idx_up = L.idx_up;
+  out->idx_down = L.idx_down;
+  out->cnt = L.cnt;
+  return WINA_OK;
+}

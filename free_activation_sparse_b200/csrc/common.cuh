@@ -1,0 +1,514 @@
+// Device building blocks shared by the kernels of the WINA sparse-linear library.
+//
+//  * element loads (bf16 / f32) and cache-hinted streaming loads of weight rows;
+//  * block-wide exclusive scan;
+//  * exact top-K by radix select on float32 score bits (scores are >= 0, so their
+//    uint32 bit patterns order like the floats), ties to the lower index;
+//  * warp-ballot compaction of a selection into an ascending index list;
+//  * a grid barrier with a time limit, for cooperative (co-resident) launches;
+//  * the split-K row accumulation of the sparse product (SVMM).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "wina.h"
+
+namespace wina {
+
+constexpr int kMaxN = 32768;                          // longest vector a gate handles in SMEM
+constexpr unsigned long long kBarrierTimeoutNs = 1000000000ull;  // 1 s per barrier wait
+
+// ------------------------------------------------------------------------------------
+// loads and status
+// ------------------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Element i of a vector stored as dtype dt, widened to float32 (exact).
+__device__ __forceinline__ float load_elem(const void* p, int dt, int64_t i) {
+  if (dt == WINA_BF16) return bf16_bits_to_f32(__ldg(reinterpret_cast<const unsigned short*>(p) + i));
+  return __ldg(reinterpret_cast<const float*>(p) + i);
+}
+
+// L2 policy: weight rows are read once per call; let them leave L2 first so that the
+// small cross-CTA buffers (partials, h) stay resident.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ uint4 ld_stream_u4(const uint4* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// First error wins; 0 means no error.
+__device__ __forceinline__ void record_status(int32_t* st, int code) {
+  if (st) atomicCAS(reinterpret_cast<int*>(st), 0, code);
+}
+
+// ------------------------------------------------------------------------------------
+// block scan
+// ------------------------------------------------------------------------------------
+
+// Exclusive prefix sum of one uint32 per thread over the block (NT a multiple of 32,
+// <= 1024). `red` is SMEM scratch of >= 32 words. Returns the thread's exclusive
+// prefix; *total (if given) receives the block total. Contains __syncthreads().
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* red, uint32_t* total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < NW ? red[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < NW) red[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const uint32_t before = warp ? red[warp - 1] : 0u;
+  if (total) *total = red[NW - 1];
+  __syncthreads();  // red may be reused right after
+  return before + x - v;
+}
+
+// ------------------------------------------------------------------------------------
+// exact top-K selection on non-negative float32 keys
+// ------------------------------------------------------------------------------------
+
+// A selection over keys: channel i is kept iff
+//     (key_i & mask) >  prefix                                  (strictly above), or
+//     (key_i & mask) == prefix and its rank among such i < r      (boundary, by index).
+// K = n is {0, 0, n}; K = 0 is {0, 0, 0}.
+struct Selection {
+  uint32_t mask, prefix, r;
+};
+
+// Radix select of the K-th largest key (1 <= K < n) over keys[0..n) in SMEM, three
+// digit passes of 12, 12 and 8 bits from the top. After each pass the digit holding
+// the K-th key is fixed; if that digit's bin holds exactly the still-needed count, all
+// of it is kept and the search stops early. `hist` is SMEM of 4096 words, `red` SMEM of
+// >= 32 words. Every thread of the block must call it.
+template <int NT>
+__device__ Selection radix_select_topk(const uint32_t* keys, int n, int K, uint32_t* hist, uint32_t* red) {
+  __shared__ uint32_t s_digit, s_rem, s_cnt;
+  uint32_t mask = 0, prefix = 0, rem = (uint32_t)K;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int sh = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
+    const int nb = pass == 2 ? 256 : 4096;
+    const uint32_t dm = (uint32_t)nb - 1u;
+    for (int i = threadIdx.x; i < nb; i += NT) hist[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += NT) {
+      const uint32_t k = keys[i];
+      if ((k & mask) == prefix) atomicAdd(&hist[(k >> sh) & dm], 1u);
+    }
+    __syncthreads();
+    // Thread t owns the bins of descending rank [t*per, (t+1)*per): bin nb-1-q for q.
+    const int per = (nb + NT - 1) / NT;
+    const int q0 = threadIdx.x * per;
+    const int q1 = min(q0 + per, nb);
+    uint32_t local = 0;
+    for (int q = q0; q < q1; ++q) local += hist[nb - 1 - q];
+    const uint32_t above = block_excl_scan<NT>(local, red, nullptr);
+    if (above < rem && above + local >= rem) {  // exactly one thread holds the crossing
+      uint32_t cum = above;
+      for (int q = q0; q < q1; ++q) {
+        const uint32_t c = hist[nb - 1 - q];
+        if (cum + c >= rem) {
+          s_digit = (uint32_t)(nb - 1 - q);
+          s_rem = rem - cum;
+          s_cnt = c;
+          break;
+        }
+        cum += c;
+      }
+    }
+    __syncthreads();
+    const uint32_t d = s_digit, cnt = s_cnt;
+    rem = s_rem;
+    prefix |= d << sh;
+    mask |= dm << sh;
+    __syncthreads();  // s_* and hist are rewritten by the next pass
+    if (cnt == rem) break;
+  }
+  return Selection{mask, prefix, rem};
+}
+
+template <int NT>
+__device__ __forceinline__ Selection select_topk_block(const uint32_t* keys, int n, int K, uint32_t* hist,
+                                                       uint32_t* red) {
+  if (K <= 0) return Selection{0u, 0u, 0u};
+  if (K >= n) return Selection{0u, 0u, (uint32_t)n};
+  return radix_select_topk<NT>(keys, n, K, hist, red);
+}
+
+// Warp-ballot compaction of a Selection, in ascending index order. Warp w walks the
+// contiguous segment [w*seg, (w+1)*seg) 32 channels at a time; a first walk counts the
+// strictly-above and boundary channels per warp, a scan over warps gives each warp its
+// bases, and a second walk computes every kept channel's output position
+//     pos(i) = #strict before i + min(#boundary before i, r).
+// emit(i, pos) is called for kept channels with lo <= pos < hi. `wsm` is SMEM of
+// >= 2*NT/32 words. Every thread of the block must call it.
+template <int NT, typename Emit>
+__device__ void compact_selection(const uint32_t* keys, int n, Selection sel, uint32_t lo, uint32_t hi, uint32_t* wsm,
+                                  Emit emit) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = (((n + NW - 1) / NW) + 31) & ~31;
+  const int b0 = warp * seg;
+  const int b1 = min(n, b0 + seg);
+  uint32_t cs = 0, ce = 0;
+  for (int base = b0; base < b1; base += 32) {
+    const int i = base + lane;
+    const bool in = i < b1;
+    const uint32_t mk = in ? (keys[i] & sel.mask) : 0u;
+    cs += __popc(__ballot_sync(0xffffffffu, in && mk > sel.prefix));
+    ce += __popc(__ballot_sync(0xffffffffu, in && mk == sel.prefix));
+  }
+  if (lane == 0) {
+    wsm[warp] = cs;
+    wsm[NW + warp] = ce;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t a = lane < NW ? wsm[lane] : 0u;
+    const uint32_t e = lane < NW ? wsm[NW + lane] : 0u;
+    uint32_t ia = a, ie = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ya = __shfl_up_sync(0xffffffffu, ia, o);
+      const uint32_t ye = __shfl_up_sync(0xffffffffu, ie, o);
+      if (lane >= o) {
+        ia += ya;
+        ie += ye;
+      }
+    }
+    if (lane < NW) {
+      wsm[lane] = ia - a;
+      wsm[NW + lane] = ie - e;
+    }
+  }
+  __syncthreads();
+  uint32_t sbase = wsm[warp], ebase = wsm[NW + warp];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = b0; base < b1; base += 32) {
+    const int i = base + lane;
+    const bool in = i < b1;
+    const uint32_t mk = in ? (keys[i] & sel.mask) : 0u;
+    const bool st = in && mk > sel.prefix;
+    const bool eq = in && mk == sel.prefix;
+    const uint32_t sb = __ballot_sync(0xffffffffu, st);
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    const uint32_t erank = ebase + __popc(eb & lt);
+    const bool keep = st || (eq && erank < sel.r);
+    const uint32_t pos = sbase + __popc(sb & lt) + min(erank, sel.r);
+    if (keep && pos >= lo && pos < hi) emit(i, pos);
+    sbase += __popc(sb);
+    ebase += __popc(eb);
+  }
+  __syncthreads();  // wsm may be reused right after
+}
+
+// Ballot compaction of a predicate (ascending index order): first counts, then calls
+// range(total, &lo, &hi) on every thread to choose the window of positions wanted, then
+// emit(i, pos) for kept channels with lo <= pos < hi. Returns the total kept count.
+template <int NT, typename Pred, typename Range, typename Emit>
+__device__ uint32_t compact_pred(int n, Pred pred, Range range, uint32_t* wsm, Emit emit) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = (((n + NW - 1) / NW) + 31) & ~31;
+  const int b0 = warp * seg;
+  const int b1 = min(n, b0 + seg);
+  uint32_t cs = 0;
+  for (int base = b0; base < b1; base += 32) {
+    const int i = base + lane;
+    cs += __popc(__ballot_sync(0xffffffffu, i < b1 && pred(i)));
+  }
+  if (lane == 0) wsm[warp] = cs;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t a = lane < NW ? wsm[lane] : 0u;
+    uint32_t ia = a;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, ia, o);
+      if (lane >= o) ia += y;
+    }
+    if (lane < NW) wsm[lane] = ia - a;
+    if (lane == NW - 1) wsm[NW] = ia;
+  }
+  __syncthreads();
+  const uint32_t total = wsm[NW];
+  uint32_t lo = 0, hi = 0;
+  range(total, &lo, &hi);
+  uint32_t sbase = wsm[warp];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = b0; base < b1; base += 32) {
+    const int i = base + lane;
+    const bool k = i < b1 && pred(i);
+    const uint32_t sb = __ballot_sync(0xffffffffu, k);
+    const uint32_t pos = sbase + __popc(sb & lt);
+    if (k && pos >= lo && pos < hi) emit(i, pos);
+    sbase += __popc(sb);
+  }
+  __syncthreads();
+  return total;
+}
+
+// ------------------------------------------------------------------------------------
+// one-pass mean / variance (Welford per thread, Chan's pairwise merge across threads)
+// ------------------------------------------------------------------------------------
+
+struct Moments {
+  double n, mean, m2;
+};
+
+__device__ __forceinline__ Moments merge_moments(Moments a, Moments b) {
+  if (b.n == 0.0) return a;
+  if (a.n == 0.0) return b;
+  const double n = a.n + b.n;
+  const double d = b.mean - a.mean;
+  return Moments{n, a.mean + d * (b.n / n), a.m2 + b.m2 + d * d * (a.n * b.n / n)};
+}
+
+// Block-wide merge in a fixed tree order (deterministic). `red` SMEM of >= 3*NT/32
+// doubles. All threads receive the result.
+template <int NT>
+__device__ Moments block_moments(Moments m, double* red) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    Moments o_;
+    o_.n = __shfl_down_sync(0xffffffffu, m.n, o);
+    o_.mean = __shfl_down_sync(0xffffffffu, m.mean, o);
+    o_.m2 = __shfl_down_sync(0xffffffffu, m.m2, o);
+    m = merge_moments(m, o_);
+  }
+  if (lane == 0) {
+    red[warp] = m.n;
+    red[NW + warp] = m.mean;
+    red[2 * NW + warp] = m.m2;
+  }
+  __syncthreads();
+  Moments t{0.0, 0.0, 0.0};
+  for (int w = 0; w < NW; ++w) t = merge_moments(t, Moments{red[w], red[NW + w], red[2 * NW + w]});
+  __syncthreads();
+  return t;
+}
+
+// ------------------------------------------------------------------------------------
+// grid barrier (cooperative launches only: all CTAs must be co-resident)
+// ------------------------------------------------------------------------------------
+
+// Lives in the caller's workspace; zero-filled before first use. `count` returns to 0
+// after every completed barrier, `gen` only grows, so the state carries over between
+// calls without a reset.
+struct GridBarrier {
+  unsigned count;
+  unsigned gen;
+  unsigned pad[30];
+};
+
+// Returns false if this CTA gave up waiting (WINA_ERR_TIMEOUT is recorded); the
+// caller must then return without touching shared results.
+__device__ __forceinline__ bool grid_sync(GridBarrier* bar, unsigned nblocks, int32_t* status) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const unsigned g0 = ld_acquire_u32(&bar->gen);
+    __threadfence();
+    const unsigned old = atomicAdd(&bar->count, 1u);
+    if (old == nblocks - 1u) {
+      atomicExch(&bar->count, 0u);
+      __threadfence();
+      atomicAdd(&bar->gen, 1u);
+    } else {
+      const unsigned long long t0 = globaltimer_ns();
+      while (ld_acquire_u32(&bar->gen) == g0) {
+        if (globaltimer_ns() - t0 > kBarrierTimeoutNs) {
+          ok = 0;
+          record_status(status, WINA_ERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// ------------------------------------------------------------------------------------
+// the sparse product's inner loop (SVMM over a CTA's share of kept rows)
+// ------------------------------------------------------------------------------------
+
+// One 16-byte vector of weights times a scalar, accumulated in float32.
+template <bool BF16>
+struct VecOps;
+
+template <>
+struct VecOps<true> {
+  static constexpr int EPV = 8;  // bf16 per 16 bytes
+  __device__ __forceinline__ static void fma(float* acc, const uint4& w, float x) {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[2 * q] = fmaf(__uint_as_float(ws[q] << 16), x, acc[2 * q]);
+      acc[2 * q + 1] = fmaf(__uint_as_float(ws[q] & 0xffff0000u), x, acc[2 * q + 1]);
+    }
+  }
+};
+
+template <>
+struct VecOps<false> {
+  static constexpr int EPV = 4;  // f32 per 16 bytes
+  __device__ __forceinline__ static void fma(float* acc, const uint4& w, float x) {
+    acc[0] = fmaf(__uint_as_float(w.x), x, acc[0]);
+    acc[1] = fmaf(__uint_as_float(w.y), x, acc[1]);
+    acc[2] = fmaf(__uint_as_float(w.z), x, acc[2]);
+    acc[3] = fmaf(__uint_as_float(w.w), x, acc[3]);
+  }
+};
+
+// Thread layout for rows of V 16-byte vectors: the block is split into NG = NT / TPR
+// groups of TPR threads; group g takes rows g, g + NG, ...; lane l of a group owns
+// vectors l, l + TPR, ..., (VPT of them).
+struct RowLayout {
+  int V;    // vectors per row
+  int TPR;  // threads per row
+  int NG;   // row groups
+  int VPT;  // vectors per thread
+};
+
+template <int NT>
+__host__ __device__ inline RowLayout make_row_layout(int64_t m, int epv) {
+  RowLayout L;
+  L.V = (int)(m / epv);
+  int t = 32;
+  while (t < L.V && t < NT) t <<= 1;
+  L.TPR = t;
+  L.NG = NT / t;
+  L.VPT = (L.V + t - 1) / t;
+  return L;
+}
+
+// acc[j][e] += sum over this group's rows r of vals[r] * Wt[rows[r]][(l + j*TPR)*EPV + e].
+// rows/vals are the CTA's share in SMEM (nrows entries). U rows are in flight at once
+// per thread (U * VPT 16-byte loads).
+template <bool BF16, int VPT, int U>
+__device__ __forceinline__ void accumulate_rows(const void* __restrict__ Wt, const RowLayout& L,
+                                                const int32_t* rows, const float* vals, int nrows,
+                                                float (&acc)[VPT][VecOps<BF16>::EPV], uint64_t pol) {
+  const int g = threadIdx.x / L.TPR;
+  const int l = threadIdx.x % L.TPR;
+  const uint4* base = reinterpret_cast<const uint4*>(Wt);
+  const int64_t V = L.V;
+  int r = g;
+  const int step = L.NG;
+  for (; r + (U - 1) * step < nrows; r += U * step) {
+    uint4 w[U][VPT];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint4* rp = base + (int64_t)rows[r + u * step] * V;
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = l + j * L.TPR;
+        if (v < L.V) w[u][j] = ld_stream_u4(rp + v, pol);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float xv = vals[r + u * step];
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        const int v = l + j * L.TPR;
+        if (v < L.V) VecOps<BF16>::fma(acc[j], w[u][j], xv);
+      }
+    }
+  }
+  for (; r < nrows; r += step) {
+    const uint4* rp = base + (int64_t)rows[r] * V;
+    const float xv = vals[r];
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = l + j * L.TPR;
+      if (v < L.V) VecOps<BF16>::fma(acc[j], ld_stream_u4(rp + v, pol), xv);
+    }
+  }
+}
+
+// Sum the NG group accumulators of a CTA and store the CTA's partial row out[0..m)
+// (float32, 16-byte aligned). With NG > 1 a row fits in one group (VPT == 1), so `red`
+// needs NG * m <= NT * EPV floats of SMEM. Deterministic: groups are added in order.
+template <bool BF16, int VPT>
+__device__ __forceinline__ void store_partial(float* __restrict__ out, const RowLayout& L,
+                                              float (&acc)[VPT][VecOps<BF16>::EPV], float* red) {
+  constexpr int EPV = VecOps<BF16>::EPV;
+  const int g = threadIdx.x / L.TPR;
+  const int l = threadIdx.x % L.TPR;
+  const int m = L.V * EPV;
+  if (L.NG == 1) {
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = l + j * L.TPR;
+      if (v < L.V) {
+        float4* o = reinterpret_cast<float4*>(out + (int64_t)v * EPV);
+#pragma unroll
+        for (int q = 0; q < EPV / 4; ++q)
+          o[q] = make_float4(acc[j][4 * q], acc[j][4 * q + 1], acc[j][4 * q + 2], acc[j][4 * q + 3]);
+      }
+    }
+    return;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int v = l + j * L.TPR;
+    if (v < L.V) {
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) red[(int64_t)g * m + v * EPV + e] = acc[j][e];
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < m; c += L.NG * L.TPR) {
+    float s = 0.f;
+    for (int gg = 0; gg < L.NG; ++gg) s += red[(int64_t)gg * m + c];
+    out[c] = s;
+  }
+  __syncthreads();
+}
+
+}  // namespace wina

@@ -1,0 +1,138 @@
+// Host-side helpers shared by the C-ABI entry points (argument checks, device facts,
+// launches, workspace layouts). Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "wina.h"
+
+namespace wina {
+
+// Largest grid any kernel here launches; workspaces are sized for it so that their
+// size does not depend on the device. (2 CTAs on each of a B200's 148 SMs.)
+constexpr int kGridCap = 296;
+constexpr int kNT = 512;          // threads per CTA of the selection / product kernels
+constexpr int kRowChunk = 1024;   // kept rows staged in SMEM at a time by sparse_matvec
+constexpr size_t kAlign = 256;    // alignment of every workspace sub-buffer
+
+inline bool valid_dtype(int dt) { return dt == WINA_F32 || dt == WINA_BF16; }
+inline int64_t elem_size(int dt) { return dt == WINA_BF16 ? 2 : 4; }
+inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline wina_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return WINA_OK;
+  return WINA_ERR_CUDA;
+}
+
+// Streaming multiprocessors of the current device (0 if none).
+int device_sm_count();
+
+// Launch with cudaLaunchKernelEx, optionally as a cooperative launch (all CTAs
+// co-resident, required by kernels that use grid_sync).
+template <typename... Exp, typename... Act>
+cudaError_t launch_kernel(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool coop,
+                          Act&&... args) {
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (coop) {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Act&&>(args)...);
+}
+
+// Largest co-resident grid for `kern` at this block size and SMEM, capped at kGridCap.
+template <typename K>
+int max_coresident_grid(K kern, int threads, size_t smem) {
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return 0;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess) return 0;
+  const int g = per_sm * device_sm_count();
+  return g < kGridCap ? g : kGridCap;
+}
+
+// ----------------------------------------------------------------------------------
+// workspace layouts
+// ----------------------------------------------------------------------------------
+
+// sparse_matvec: [GridBarrier][partials: kGridCap x m float32]. Only needed when a
+// token is split over several CTAs (batch < kGridCap).
+struct SpmvWs {
+  size_t bar, partials, total;
+};
+inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
+  SpmvWs w;
+  w.bar = 0;
+  w.partials = kAlign;
+  const size_t part = batch < kGridCap ? (size_t)kGridCap * (size_t)m * 4 : 0;
+  w.total = round_up(w.partials + part, kAlign);
+  return w;
+}
+
+// sparse_ffn_swiglu (d, ffn, batch):
+//   bar | h [B][ffn] | keys_d [B][ffn] | idx_gate [B][d] | idx_up [B][d] | idx_down [B][ffn]
+//   | cnt [3][B] | xs_gate [B][d] | xs_up [B][d] | xs_down [B][ffn] | g [B][ffn] | u [B][ffn]
+//   | part_g [kGridCap][ffn] | part_u [kGridCap][ffn] | part_d [kGridCap][d] | spmv ws
+struct FfnWs {
+  size_t bar, h, keys_d, idx_gate, idx_up, idx_down, cnt, xs_gate, xs_up, xs_down, g, u, part_g, part_u, part_d,
+      spmv, total;
+};
+inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
+  FfnWs w;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = round_up(o + bytes, kAlign);
+    return at;
+  };
+  w.bar = take(sizeof(GridBarrier));
+  w.h = take((size_t)B * ffn * 4);
+  w.keys_d = take((size_t)B * ffn * 4);
+  w.idx_gate = take((size_t)B * d * 4);
+  w.idx_up = take((size_t)B * d * 4);
+  w.idx_down = take((size_t)B * ffn * 4);
+  w.cnt = take((size_t)3 * B * 4);
+  w.xs_gate = take((size_t)B * d * 4);
+  w.xs_up = take((size_t)B * d * 4);
+  w.xs_down = take((size_t)B * ffn * 4);
+  w.g = take((size_t)B * ffn * 4);
+  w.u = take((size_t)B * ffn * 4);
+  const size_t gp = (size_t)kGridCap * ffn * 4, dp = (size_t)kGridCap * d * 4;
+  w.part_g = take(B == 1 ? gp : 0);
+  w.part_u = take(B == 1 ? gp : 0);
+  w.part_d = take(B == 1 ? dp : 0);
+  const int64_t mmax = ffn > d ? ffn : d;
+  w.spmv = take(B == 1 ? 0 : spmv_ws_layout(mmax, B).total);
+  w.total = o;
+  return w;
+}
+
+// ----------------------------------------------------------------------------------
+// launchers implemented in the kernel files (arguments already checked)
+// ----------------------------------------------------------------------------------
+
+wina_status_t launch_select_topk(const void* x, int xdt, const float* c, int n, int k, int batch, int32_t* idx,
+                                 float* xs, int ld, float* scores, cudaStream_t s);
+wina_status_t launch_stat_threshold(const void* v, int vdt, int n, double z, int batch, int32_t* idx, float* xs,
+                                    int32_t* count, float* t, int cap, int32_t* status_dev, cudaStream_t s);
+wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx,
+                                   const float* xs, int k, const int32_t* count, int ld_idx, int batch, float* y,
+                                   void* ws, int32_t* status_dev, cudaStream_t s);
+wina_status_t launch_silu_mul(const float* g, const float* u, float* h, int64_t count, cudaStream_t s);
+
+}  // namespace wina

@@ -1,0 +1,126 @@
+// Per-token gates: the WINA top-K gate and the Spark statistical threshold.
+//
+//  * wina_select_topk ("WINA" article, section 一): score_i = |x_i * c_i| in float32,
+//    keep the K largest (ties to the lower index), written as an ascending index list.
+//    One CTA per token: scores live in SMEM as uint32 bit patterns, a three-pass radix
+//    select finds the K-th largest, a two-walk warp-ballot compaction emits the list.
+//  * stat_topk_threshold ("Spark Transformer", section 2.2): mu, sigma^2 (divisor n) in
+//    one pass (Welford per thread, Chan's merge across threads, float64), then
+//    t = mu + sigma * z with z = Phi^-1(1 - s) from the host, keep {i : v_i > t}.
+#include <math.h>
+
+#include "internal.h"
+
+namespace wina {
+
+template <int NT>
+__global__ void __launch_bounds__(NT) k_select_topk(const void* __restrict__ x, int xdt, const float* __restrict__ c,
+                                                    int n, int K, int ld, int32_t* __restrict__ idx,
+                                                    float* __restrict__ xs, float* __restrict__ scores) {
+  extern __shared__ __align__(16) uint32_t sm[];
+  uint32_t* keys = sm;       // [n]
+  uint32_t* hist = sm + n;   // [4096]
+  __shared__ uint32_t red[64];
+  const int64_t b = blockIdx.x;
+  const int64_t off = b * (int64_t)n;
+  for (int i = threadIdx.x; i < n; i += NT) {
+    const float xv = load_elem(x, xdt, off + i);
+    const float s = c ? fabsf(xv * __ldg(c + i)) : fabsf(xv);
+    keys[i] = __float_as_uint(s);
+    if (scores) scores[off + i] = s;
+  }
+  __syncthreads();
+  const Selection sel = select_topk_block<NT>(keys, n, K, hist, red);
+  const int64_t ob = b * (int64_t)ld;
+  compact_selection<NT>(keys, n, sel, 0u, (uint32_t)K, red, [&](int i, uint32_t pos) {
+    idx[ob + pos] = i;
+    if (xs) xs[ob + pos] = load_elem(x, xdt, off + i);
+  });
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) k_stat_threshold(const void* __restrict__ v, int vdt, int n, double z,
+                                                       int32_t* __restrict__ idx, float* __restrict__ xs,
+                                                       int32_t* __restrict__ count, float* __restrict__ tout, int cap,
+                                                       int32_t* status) {
+  extern __shared__ __align__(16) float vals[];  // [n]
+  __shared__ double dred[3 * NT / 32];
+  __shared__ uint32_t wsm[2 * NT / 32 + 1];
+  const int64_t b = blockIdx.x;
+  const int64_t off = b * (int64_t)n;
+  Moments mo{0.0, 0.0, 0.0};
+  for (int i = threadIdx.x; i < n; i += NT) {
+    const float f = load_elem(v, vdt, off + i);
+    vals[i] = f;
+    mo.n += 1.0;
+    const double dl = (double)f - mo.mean;
+    mo.mean += dl / mo.n;
+    mo.m2 += dl * ((double)f - mo.mean);
+  }
+  const Moments tot = block_moments<NT>(mo, dred);  // contains __syncthreads
+  const double mu = tot.mean;
+  const double var = tot.m2 / (double)n;
+  const double t = mu + sqrt(var) * z;
+  const int64_t ob = b * (int64_t)cap;
+  const uint32_t total = compact_pred<NT>(
+      n, [&](int i) { return (double)vals[i] > t; },
+      [&](uint32_t, uint32_t* lo, uint32_t* hi) {
+        *lo = 0;
+        *hi = (uint32_t)cap;
+      },
+      wsm,
+      [&](int i, uint32_t pos) {
+        idx[ob + pos] = i;
+        if (xs) xs[ob + pos] = vals[i];
+      });
+  if (threadIdx.x == 0) {
+    count[b] = (int32_t)total;
+    if (tout) tout[b] = (float)t;
+    if ((int64_t)total > cap) record_status(status, WINA_ERR_CAPACITY);
+  }
+}
+
+wina_status_t launch_select_topk(const void* x, int xdt, const float* c, int n, int k, int batch, int32_t* idx,
+                                 float* xs, int ld, float* scores, cudaStream_t s) {
+  const size_t smem = (size_t)(n + 4096) * 4;
+  return cuda_status(launch_kernel(k_select_topk<kNT>, dim3(batch), dim3(kNT), smem, s, false, x, xdt, c, n, k, ld,
+                                   idx, xs, scores));
+}
+
+wina_status_t launch_stat_threshold(const void* v, int vdt, int n, double z, int batch, int32_t* idx, float* xs,
+                                    int32_t* count, float* t, int cap, int32_t* status_dev, cudaStream_t s) {
+  const size_t smem = (size_t)n * 4;
+  return cuda_status(launch_kernel(k_stat_threshold<kNT>, dim3(batch), dim3(kNT), smem, s, false, v, vdt, n, z, idx,
+                                   xs, count, t, cap, status_dev));
+}
+
+}  // namespace wina
+
+using namespace wina;
+
+extern "C" wina_status_t wina_select_topk(const void* x, wina_dtype_t xdt, const float* c, int64_t n, int64_t k,
+                                          int64_t batch, int32_t* idx, float* xs, float* scores,
+                                          wina_stream_t stream) {
+  if (!valid_dtype(xdt)) return WINA_ERR_UNSUPPORTED_DTYPE;
+  if (n < 1 || n > kMaxN || k < 0 || k > n || batch < 1 || batch > INT32_MAX) return WINA_ERR_INVALID_ARG;
+  if (!x || (k > 0 && !idx)) return WINA_ERR_INVALID_ARG;
+  if (!aligned(x, elem_size(xdt)) || (c && !aligned(c, 4)) || (idx && !aligned(idx, 4)) || (xs && !aligned(xs, 4)) ||
+      (scores && !aligned(scores, 4)))
+    return WINA_ERR_INVALID_ARG;
+  return launch_select_topk(x, xdt, c, (int)n, (int)k, (int)batch, idx, xs, (int)k, scores, (cudaStream_t)stream);
+}
+
+extern "C" wina_status_t stat_topk_threshold(const void* v, wina_dtype_t vdt, int64_t n, double s, int64_t batch,
+                                             int32_t* idx, float* xs, int32_t* count, float* t, int64_t cap,
+                                             int32_t* status_dev, wina_stream_t stream) {
+  if (!valid_dtype(vdt)) return WINA_ERR_UNSUPPORTED_DTYPE;
+  if (n < 1 || n > kMaxN || batch < 1 || batch > INT32_MAX || cap < 0 || cap > INT32_MAX) return WINA_ERR_INVALID_ARG;
+  if (!(s > 0.0 && s < 1.0)) return WINA_ERR_INVALID_ARG;
+  if (!v || !count || (cap > 0 && !idx)) return WINA_ERR_INVALID_ARG;
+  if (!aligned(v, elem_size(vdt)) || !aligned(count, 4) || (idx && !aligned(idx, 4)) || (xs && !aligned(xs, 4)) ||
+      (t && !aligned(t, 4)) || (status_dev && !aligned(status_dev, 4)))
+    return WINA_ERR_INVALID_ARG;
+  const double z = wina_normal_quantile(1.0 - s);
+  return launch_stat_threshold(v, vdt, (int)n, z, (int)batch, idx, xs, count, t, (int)cap, status_dev,
+                               (cudaStream_t)stream);
+}

@@ -1,0 +1,239 @@
+/*
+ * wina.h -- C ABI of the weight-informed, activation-sparse linear layer for LLM decode
+ * (CUDA, sm_100a / B200).
+ *
+ * The method (WINA gate):
+ *   offline:   c_j = || W[:, j] ||_2, the l2 norm of each input column of W [out][in];
+ *   per token: score_i = | x_i * c_i |, keep the K largest (ties -> lower index), or,
+ *              in the Spark variant, keep { i : v_i > mu + sigma * Phi^-1(1 - s) };
+ *              y = W[:, S] x[S], reading only the kept columns of W.
+ * Sources, cited by page title and section:
+ *   - "WINA: Weight Informed Neuron Activation" article (lsdiaocha.cn, 2025-05-29),
+ *     section 一 (the gate: top-K of |x (.) c| with c the column l2 norms of W; K may be
+ *     shared or per layer), section 二 (error bound for column-orthogonal W);
+ *   - "Spark Transformer: 高效稀疏化大语言模型架构设计", section 2.2 (statistical top-k:
+ *     mean, population variance, Gaussian quantile threshold, strict comparison) and
+ *     section 3.1 (SVMM: accumulate x_j * W[j] over the active indices only, with W
+ *     stored input-major so that W[j] is one contiguous run);
+ *   - "哈工大EMNLP 2025论文开源 ... WAS", section on the core innovations (the gate is
+ *     applied per component: Q, K, V, O, gate, up and down projections).
+ *
+ * Conventions (every call):
+ *   - Returns wina_status_t; WINA_OK is 0. Arguments are checked on the host before any
+ *     launch; a bad argument returns an error code and launches nothing.
+ *   - Every pointer argument except those documented as host pointers is a DEVICE
+ *     pointer, allocated and owned by the caller. The library allocates no device or
+ *     host memory and keeps no state between calls (see wina_workspace_size for the
+ *     scratch a call needs). Device pointers must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     Launch errors are returned at once (WINA_ERR_CUDA). Errors found on the device
+ *     (capacity overflow, a grid-barrier timeout) are written into the optional
+ *     caller-owned int32 word `status_dev` (first error wins; 0 = none) and are seen by
+ *     the caller after it synchronises. Pass NULL to ignore them.
+ *   - Weights are stored input-channel-major: Wt[n][m] = W[m][n]^T, so input channel j
+ *     is the contiguous run Wt[j][0..m). wina_pack_in_major produces this layout.
+ *   - dtype: WINA_BF16 (bfloat16) or WINA_F32. Products accumulate in float32; outputs y
+ *     are float32.
+ *   - Inputs must be finite; NaN/Inf inputs are not supported (results unspecified).
+ */
+#ifndef WINA_H
+#define WINA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WINA_ABI_VERSION 1
+
+/* A cudaStream_t, declared opaquely so this header does not need the CUDA headers. */
+typedef struct CUstream_st* wina_stream_t;
+
+typedef enum {
+  WINA_OK = 0,
+  WINA_ERR_INVALID_ARG = 1,       /* bad size, null or misaligned pointer, k > n, s outside (0,1) */
+  WINA_ERR_UNSUPPORTED_DTYPE = 2, /* dtype not in {WINA_F32, WINA_BF16} */
+  WINA_ERR_WORKSPACE = 3,         /* workspace smaller than wina_workspace_size() */
+  WINA_ERR_CAPACITY = 4,          /* device: more channels passed the threshold than `cap` */
+  WINA_ERR_CUDA = 5,              /* a CUDA runtime call failed (no device, launch error) */
+  WINA_ERR_TIMEOUT = 6            /* device: a grid-barrier wait gave up after its time limit */
+} wina_status_t;
+
+typedef enum { WINA_F32 = 0, WINA_BF16 = 1 } wina_dtype_t;
+
+/* Memory layout of a weight passed to wina_col_norms. */
+typedef enum {
+  WINA_LAYOUT_OUT_IN = 0, /* W[m][n]: row i is output i (the matrix that multiplies x)   */
+  WINA_LAYOUT_IN_MAJOR = 1 /* Wt[n][m]: row j is input channel j (the packed layout)     */
+} wina_layout_t;
+
+/* How sparse_ffn_swiglu chooses the kept channels of each projection's input. */
+typedef enum {
+  WINA_GATE_TOPK = 0,  /* WINA: top-K of |v_i * c_i| with the projection's own c and K */
+  WINA_GATE_STAT = 1,  /* Spark: { i : v_i > mu + sigma * Phi^-1(1 - s) } on the signed v */
+  WINA_GATE_DENSE = 2  /* no gate: every channel is kept (the dense comparator)          */
+} wina_gate_mode_t;
+
+typedef enum {
+  WINA_OP_SELECT_TOPK = 0,
+  WINA_OP_STAT_THRESHOLD = 1,
+  WINA_OP_SPARSE_MATVEC = 2,
+  WINA_OP_FFN_SWIGLU = 3
+} wina_op_t;
+
+/* The three projections of a SwiGLU FFN, already packed input-major:
+ *   wt_gate, wt_up: [d][ffn];  wt_down: [ffn][d];  all of dtype wdt.
+ *   c_gate, c_up: float32 [d];  c_down: float32 [ffn]  (column norms of W_gate, W_up,
+ *   W_down, as written by wina_col_norms). Only WINA_GATE_TOPK reads the c's. */
+typedef struct {
+  const void* wt_gate;
+  const void* wt_up;
+  const void* wt_down;
+  wina_dtype_t wdt;
+  const float* c_gate;
+  const float* c_up;
+  const float* c_down;
+  int64_t d;
+  int64_t ffn;
+} wina_ffn_t;
+
+/* Byte offsets, inside the workspace of a sparse_ffn_swiglu call, of the intermediate
+ * results it leaves behind (valid after the call completes; read-only diagnostics):
+ *   h        float32 [batch][ffn]   h = silu(g) * u, the down projection's input
+ *   idx_gate int32  [batch][d]      kept gate channels, ascending (first cnt_gate[b])
+ *   idx_up   int32  [batch][d]      kept up channels, ascending
+ *   idx_down int32  [batch][ffn]    kept down channels, ascending
+ *   cnt      int32  [3][batch]      kept counts of gate, up and down per token        */
+typedef struct {
+  size_t h;
+  size_t idx_gate;
+  size_t idx_up;
+  size_t idx_down;
+  size_t cnt;
+} wina_ffn_ws_view_t;
+
+/* ABI version of the loaded library (WINA_ABI_VERSION at build time). */
+int32_t wina_abi_version(void);
+
+/* Static description of a status code (host pointer to a constant string). */
+const char* wina_status_string(wina_status_t status);
+
+/* Standard normal quantile Phi^-1(p) for 0 < p < 1, in double precision (host function;
+ * no device needed). The Spark threshold uses z = Phi^-1(1 - s) ("Spark Transformer",
+ * section 2.2: Phi is the standard normal CDF). Computed by Newton iteration on
+ * Phi(z) = erfc(-z / sqrt 2) / 2 from a bracketing start; |error| ~ 1e-15.
+ * Returns NaN for p outside (0, 1). */
+double wina_normal_quantile(double p);
+
+/* Bytes of device scratch that `op` needs for the given sizes (0 if none). The
+ * workspace is owned by the caller, must be zero-filled before its first use, and may
+ * be reused by later calls of the same op on the same stream; the library leaves it in
+ * a reusable state unless a call ended in WINA_ERR_TIMEOUT, after which it must be
+ * zero-filled again. Concurrent calls need distinct workspaces.
+ *   WINA_OP_SPARSE_MATVEC: n = in-features, m = out-features, k = max kept per token,
+ *                          batch = tokens.
+ *   WINA_OP_FFN_SWIGLU:    n = d, m = ffn, k ignored, batch = tokens.
+ *   WINA_OP_SELECT_TOPK, WINA_OP_STAT_THRESHOLD: 0.                                  */
+size_t wina_workspace_size(wina_op_t op, int64_t n, int64_t m, int64_t k, int64_t batch);
+
+/* Offsets of the diagnostic views inside a sparse_ffn_swiglu workspace (host function).
+ * Returns WINA_ERR_INVALID_ARG for non-positive sizes or a null `out`. */
+wina_status_t wina_ffn_ws_view(int64_t d, int64_t ffn, int64_t batch, wina_ffn_ws_view_t* out);
+
+/* Offline: transpose W[m][n] (output-major, the matrix that multiplies x) into the
+ * input-channel-major Wt[n][m] used by every product below ("Spark Transformer",
+ * section 3.1: SVMM reads W[j] as a whole for each active j). Bit-exact copy.
+ *   W:  device, m*n elements of dt, row-major [m][n];  Wt: device, [n][m], same dtype.
+ *   m, n >= 1. W and Wt must not overlap. */
+wina_status_t wina_pack_in_major(const void* W, wina_dtype_t dt, int64_t m, int64_t n, void* Wt,
+                                 wina_stream_t stream);
+
+/* Offline: column l2 norms c_j = sqrt(sum_i W[i][j]^2) for j < n ("WINA" article,
+ * section 一: c holds the l2 norm of each column of W). Squares are summed in float64,
+ * the square root is taken in float64 and rounded once to float32.
+ *   W: device; layout WINA_LAYOUT_OUT_IN means W[m][n]; WINA_LAYOUT_IN_MAJOR means the
+ *      packed Wt[n][m] (the norm of row j of Wt). m = out-features, n = in-features.
+ *   c: device float32 [n] (written). */
+wina_status_t wina_col_norms(const void* W, wina_dtype_t dt, int64_t m, int64_t n, wina_layout_t layout,
+                             float* c, wina_stream_t stream);
+
+/* Per-token top-K gate ("WINA" article, section 一): for each of `batch` tokens,
+ * score_i = |x_i * c_i| (one float32 multiply; c == NULL gives the magnitude-only gate
+ * |x_i| of TEAL/CATS), keep the k largest scores, ties at the k-th value to the lower
+ * index.
+ *   x:      device [batch][n] of xdt;  c: device float32 [n] or NULL.
+ *   idx:    device int32 [batch][k]: kept indices of each token, ascending.
+ *   xs:     device float32 [batch][k] or NULL: x at the kept indices (the stored value,
+ *           widened to float32), in the order of idx.
+ *   scores: device float32 [batch][n] or NULL: the score vector.
+ *   1 <= n <= 32768, 0 <= k <= n, batch >= 1. */
+wina_status_t wina_select_topk(const void* x, wina_dtype_t xdt, const float* c, int64_t n, int64_t k,
+                               int64_t batch, int32_t* idx, float* xs, float* scores, wina_stream_t stream);
+
+/* Spark statistical top-k ("Spark Transformer", section 2.2) for each of `batch`
+ * vectors v_b of length n: mu = mean(v), sigma^2 = mean((v - mu)^2) (divisor n),
+ * t = mu + sigma * Phi^-1(1 - s), keep { i : v_i > t } (strict, signed). The mean and
+ * variance are accumulated in float64 in one pass (per-thread Welford, Chan's pairwise
+ * merge across threads); the comparison is made in float64.
+ *   v:     device [batch][n] of vdt.   s: keep fraction, 0 < s < 1.
+ *   idx:   device int32 [batch][cap]: kept indices ascending (the first min(count, cap)).
+ *   xs:    device float32 [batch][cap] or NULL: v at the kept indices.
+ *   count: device int32 [batch]: the true number of kept channels (may exceed cap).
+ *   t:     device float32 [batch] or NULL: the threshold, rounded to float32.
+ *   cap >= 0. If a count exceeds cap only cap indices are written and WINA_ERR_CAPACITY
+ *   is recorded in *status_dev. 1 <= n <= 32768. */
+wina_status_t stat_topk_threshold(const void* v, wina_dtype_t vdt, int64_t n, double s, int64_t batch,
+                                  int32_t* idx, float* xs, int32_t* count, float* t, int64_t cap,
+                                  int32_t* status_dev, wina_stream_t stream);
+
+/* Sparse product over the kept channels ("Spark Transformer", section 3.1, SVMM):
+ *   y[b][:] = sum over r < k_b of xs[b][r] * Wt[idx[b][r]][:]      for b < batch,
+ * reading only the kept rows of the input-major weight. One token (batch == 1) is
+ * split across all SMs by kept rows (split-K) with a deterministic reduction; several
+ * tokens are served from the union of their kept rows, each row read once per call.
+ *   Wt:    device [n][m] of wdt (m % 8 == 0 and m <= 32768 for bf16; m % 4 == 0 and
+ *          m <= 16384 for f32).
+ *   idx:   device int32 [batch][ld_idx]: kept input channels of each token (any order;
+ *          distinct within a token; each < n).
+ *   xs:    device float32 [batch][ld_idx]: the input values at those channels.
+ *   k:     kept count of every token (0 <= k <= ld_idx), or -1 to read each token's
+ *          count from the device array `count` [batch] (as written by
+ *          stat_topk_threshold; counts above ld_idx are clamped to ld_idx).
+ *   y:     device float32 [batch][m] (written; does not alias the inputs).
+ *   ws:    device scratch of at least wina_workspace_size(WINA_OP_SPARSE_MATVEC, n, m,
+ *          ld_idx, batch) bytes (see that function for its lifetime rules).
+ *   status_dev: optional device int32 word for WINA_ERR_TIMEOUT. */
+wina_status_t sparse_matvec(const void* Wt, wina_dtype_t wdt, int64_t n, int64_t m, const int32_t* idx,
+                            const float* xs, int64_t k, const int32_t* count, int64_t ld_idx, int64_t batch,
+                            float* y, void* ws, size_t ws_bytes, int32_t* status_dev, wina_stream_t stream);
+
+/* SwiGLU FFN decode with the gate on every projection ("WAS" article: the gate is
+ * applied per component, gate/up/down among them; "WINA" article, section 一: each
+ * projection uses the column norms of its own weight and its own K):
+ *   S_g = gate(x, c_gate, k_gate);  g = W_gate[:, S_g] x[S_g]
+ *   S_u = gate(x, c_up,   k_up);    u = W_up[:, S_u]   x[S_u]
+ *   h   = silu(g) * u                (float32; silu(g) = g / (1 + e^-g))
+ *   S_d = gate(h, c_down, k_down);  y = W_down[:, S_d] h[S_d]
+ * With WINA_GATE_STAT every gate is the Spark threshold with keep fraction s on the
+ * projection's signed input (k_* ignored); with WINA_GATE_DENSE every channel is kept.
+ * One token runs as one persistent cooperative kernel (every SM selects redundantly
+ * from x, streams its share of kept rows, and grid barriers separate the phases);
+ * several tokens run as a sequence of the batched calls above.
+ *   f:   host pointer to the weight descriptor (read during the call only).
+ *   x:   device [batch][d] of xdt.   y: device float32 [batch][d] (written).
+ *   k_gate, k_up in [0, d]; k_down in [0, ffn] (WINA_GATE_TOPK).  0 < s < 1 (STAT).
+ *   ws:  device scratch of at least wina_workspace_size(WINA_OP_FFN_SWIGLU, d, ffn, 0,
+ *        batch) bytes; after the call it holds the views of wina_ffn_ws_view.
+ *   d % 8 == 0 and ffn % 8 == 0 (bf16) or % 4 (f32); d, ffn <= 32768 (bf16) or
+ *   <= 16384 (f32). */
+wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, wina_dtype_t xdt, int64_t batch,
+                                wina_gate_mode_t mode, int64_t k_gate, int64_t k_up, int64_t k_down, double s,
+                                float* y, void* ws, size_t ws_bytes, int32_t* status_dev, wina_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WINA_H */

@@ -1,0 +1,185 @@
+"""GPU parity of the gated SwiGLU FFN (sparse_ffn_swiglu) against the CPU oracle.
+
+Checked stage by stage on the intermediate results the call leaves in its workspace:
+  gate/up kept sets   == oracle top-K of |x * c| (bit-exact; same x and c),
+  h                   ~= oracle h from those sets (rel-L2 <= 1e-5),
+  down kept set       == oracle top-K of |h_gpu * c_down| (bit-exact on the GPU's h),
+  y                   ~= oracle product over the GPU's down set and h (rel-L2 <= 1e-5),
+and end to end: y ~= the pure float64 oracle FFN, rel-L2 <= 5e-3 (the stated bar;
+near-threshold swaps in the down set are allowed there).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle as O
+import synth
+import free_activation_sparse_b200 as W
+from tests.gpu_util import dev_bf16, dev_f32, host, rel_l2, status_word
+
+pytestmark = pytest.mark.gpu
+
+TOL_E2E = 5e-3
+TOL_STAGE = 1e-5
+
+
+def _prep_bf16(Wg, Wu, Wd):
+    return W.ffn_prepare(dev_bf16(Wg), dev_bf16(Wu), dev_bf16(Wd))
+
+
+def _check_topk_ffn(f, Wgf, Wuf, Wdf, xb, x32, kg, ku, kd, batch=None):
+    """x32 [B][d] float32 values of the input; xb the device tensor."""
+    B, d = x32.shape
+    ffn = Wgf.shape[0]
+    cg, cu, cd = host(f.c_gate), host(f.c_up), host(f.c_down)
+    st = status_word()
+    ws = W.Workspace(W.OP_FFN_SWIGLU, d, ffn, 0, B)
+    y = host(W.sparse_ffn_swiglu(f, xb, W.GATE_TOPK, kg, ku, kd, ws=ws, status=st))
+    assert int(host(st)[0]) == 0
+    v = {k: host(t) for k, t in W.ffn_ws_view(ws, d, ffn, B).items()}
+    for b in range(B):
+        ig = O.wina_select(x32[b], cg, kg)
+        iu = O.wina_select(x32[b], cu, ku)
+        assert np.array_equal(v["idx_gate"][b][:kg], ig)
+        assert np.array_equal(v["idx_up"][b][:ku], iu)
+        x64 = x32[b].astype(np.float64)
+        h_ref = O.silu(O.sparse_matvec(Wgf, ig, x64[ig])) * O.sparse_matvec(Wuf, iu, x64[iu])
+        h_gpu = v["h"][b]
+        assert rel_l2(h_gpu, h_ref) <= TOL_STAGE
+        idn = O.wina_select(h_gpu, cd, kd)
+        assert np.array_equal(v["idx_down"][b][:kd], idn)
+        assert rel_l2(y[b], O.sparse_matvec(Wdf, idn, h_gpu[idn].astype(np.float64))) <= TOL_STAGE
+        e2e = O.ffn_swiglu(Wgf, Wuf, Wdf, cg, cu, cd, x32[b], kg, ku, kd)
+        assert rel_l2(y[b], e2e["y"]) <= TOL_E2E
+    if B == 1:
+        assert v["cnt"][:, 0].tolist() == [kg, ku, kd]
+    return y
+
+
+@pytest.fixture(scope="module")
+def llama7b():
+    cfg = synth.make_llama7b_ffn(batch=4)
+    f = _prep_bf16(cfg["Wg"], cfg["Wu"], cfg["Wd"])
+    Wgf, Wuf, Wdf = (O.widen_bf16(cfg[k]) for k in ("Wg", "Wu", "Wd"))
+    return cfg, f, Wgf, Wuf, Wdf
+
+
+def test_llama7b_norms_bit_exact(llama7b):
+    cfg, f, Wgf, Wuf, Wdf = llama7b
+    assert np.array_equal(host(f.c_gate), O.col_norms(Wgf))
+    assert np.array_equal(host(f.c_up), O.col_norms(Wuf))
+    assert np.array_equal(host(f.c_down), O.col_norms(Wdf))
+
+
+@pytest.mark.parametrize("p", [0.5, 0.65])
+def test_llama7b_fused_single_token(llama7b, p):
+    cfg, f, Wgf, Wuf, Wdf = llama7b
+    d, ffn = cfg["d"], cfg["ffn"]
+    kg, kd = synth.keep_count(p, d), synth.keep_count(p, ffn)
+    xb = cfg["x"][:1]
+    _check_topk_ffn(f, Wgf, Wuf, Wdf, dev_bf16(xb), synth.f32_from_bf16_bits(xb), kg, kg, kd)
+
+
+def test_llama7b_batched_tokens(llama7b):
+    cfg, f, Wgf, Wuf, Wdf = llama7b
+    kg, kd = cfg["k_gate"], cfg["k_down"]
+    xb = cfg["x"]
+    _check_topk_ffn(f, Wgf, Wuf, Wdf, dev_bf16(xb), synth.f32_from_bf16_bits(xb), kg, kg, kd)
+
+
+def test_llama7b_extreme_k(llama7b):
+    cfg, f, Wgf, Wuf, Wdf = llama7b
+    xb = cfg["x"][:1]
+    x32 = synth.f32_from_bf16_bits(xb)
+    _check_topk_ffn(f, Wgf, Wuf, Wdf, dev_bf16(xb), x32, 1, 4096, 11007)
+    _check_topk_ffn(f, Wgf, Wuf, Wdf, dev_bf16(xb), x32, 4096, 7, 1)
+
+
+def test_llama7b_k_zero_gives_zero(llama7b):
+    cfg, f, *_ = llama7b
+    y = host(W.sparse_ffn_swiglu(f, dev_bf16(cfg["x"][:1]), W.GATE_TOPK, 0, 2048, 5504))
+    assert not y.any()  # g = 0 -> silu(0) = 0 -> h = 0 -> y = 0
+
+
+def test_llama7b_dense_mode(llama7b):
+    cfg, f, Wgf, Wuf, Wdf = llama7b
+    xb = cfg["x"][:1]
+    x32 = synth.f32_from_bf16_bits(xb)[0]
+    y = host(W.sparse_ffn_swiglu(f, dev_bf16(xb), W.GATE_DENSE))
+    x64 = x32.astype(np.float64)
+    h = O.silu(O.dense_matvec(Wgf, x64)) * O.dense_matvec(Wuf, x64)
+    assert rel_l2(y[0], O.dense_matvec(Wdf, h)) <= 1e-5
+
+
+def test_llama7b_deterministic(llama7b):
+    cfg, f, *_ = llama7b
+    ws = W.Workspace(W.OP_FFN_SWIGLU, 4096, 11008, 0, 1)
+    xb = dev_bf16(cfg["x"][:1])
+    a = host(W.sparse_ffn_swiglu(f, xb, W.GATE_TOPK, 2048, 2048, 5504, ws=ws))
+    for _ in range(3):
+        assert np.array_equal(a, host(W.sparse_ffn_swiglu(f, xb, W.GATE_TOPK, 2048, 2048, 5504, ws=ws)))
+
+
+@pytest.mark.parametrize("d,ffn,dt", [(64, 128, "bf16"), (512, 1024, "f32"), (2304, 9216, "bf16"), (8, 16, "f32")])
+def test_small_and_odd_shapes(d, ffn, dt):
+    rng = np.random.default_rng(d + ffn)
+    Wg = synth.make_weight(rng, ffn, d, 0.02, dt)
+    Wu = synth.make_weight(rng, ffn, d, 0.02, dt)
+    Wd = synth.make_weight(rng, d, ffn, 0.02, dt)
+    x = rng.laplace(size=(1, d)).astype(np.float32)
+    if dt == "bf16":
+        f = _prep_bf16(Wg, Wu, Wd)
+        Wgf, Wuf, Wdf = (O.widen_bf16(a) for a in (Wg, Wu, Wd))
+    else:
+        f = W.ffn_prepare(dev_f32(Wg), dev_f32(Wu), dev_f32(Wd))
+        Wgf, Wuf, Wdf = (a.astype(np.float64) for a in (Wg, Wu, Wd))
+    for B in (1, 3):
+        xs = np.repeat(x, B, axis=0) if B > 1 else x
+        xs = xs + np.arange(B, dtype=np.float32)[:, None] * 0.01
+        _check_topk_ffn(f, Wgf, Wuf, Wdf, dev_f32(xs), xs, d // 2, d // 3 + 1, ffn // 2 + 1)
+
+
+# ------------------------------------------------------------------------------------
+# Spark statistical gate inside the FFN (Gemma-2-2B shapes)
+# ------------------------------------------------------------------------------------
+
+
+@pytest.fixture(scope="module")
+def gemma():
+    cfg = synth.make_gemma2_2b_spark(batch=8)
+    f = _prep_bf16(cfg["Wg"], cfg["Wu"], cfg["Wd"])
+    Wgf, Wuf, Wdf = (O.widen_bf16(cfg[k]) for k in ("Wg", "Wu", "Wd"))
+    return cfg, f, Wgf, Wuf, Wdf
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_gemma_stat_gate(gemma, B):
+    cfg, f, Wgf, Wuf, Wdf = gemma
+    d, ffn, s = cfg["d"], cfg["ffn"], cfg["s"]
+    xb = cfg["x_bf16"][:B]
+    x32 = synth.f32_from_bf16_bits(xb)
+    ws = W.Workspace(W.OP_FFN_SWIGLU, d, ffn, 0, B)
+    st = status_word()
+    y = host(W.sparse_ffn_swiglu(f, dev_bf16(xb), W.GATE_STAT, s=s, ws=ws, status=st))
+    assert int(host(st)[0]) == 0
+    v = {k: host(t) for k, t in W.ffn_ws_view(ws, d, ffn, B).items()}
+    cnt = v["cnt"]
+    for b in range(B):
+        ref = O.spark_threshold(x32[b], s)
+        ig = v["idx_gate"][b][: cnt[0][b]]
+        diff = np.setxor1d(ig, ref["idx"])
+        assert np.all(np.abs(x32[b][diff] - ref["t"]) <= 1e-5 * ref["sigma"])
+        assert np.array_equal(v["idx_up"][b][: cnt[1][b]], ig)
+        x64 = x32[b].astype(np.float64)
+        h_ref = O.silu(O.sparse_matvec(Wgf, ig, x64[ig])) * O.sparse_matvec(Wuf, ig, x64[ig])
+        h_gpu = v["h"][b]
+        assert rel_l2(h_gpu, h_ref) <= TOL_STAGE
+        rd = O.spark_threshold(h_gpu, s)
+        idn = v["idx_down"][b][: cnt[2][b]]
+        diff = np.setxor1d(idn, rd["idx"])
+        assert np.all(np.abs(h_gpu[diff] - rd["t"]) <= 1e-5 * rd["sigma"])
+        assert rel_l2(y[b], O.sparse_matvec(Wdf, idn, h_gpu[idn].astype(np.float64))) <= TOL_STAGE
+        e2e = O.ffn_swiglu(Wgf, Wuf, Wdf, None, None, None, x32[b], 0, 0, 0, mode="stat", s=s)
+        assert rel_l2(y[b], e2e["y"]) <= TOL_E2E
