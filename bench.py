@@ -233,24 +233,47 @@ def main():
             if ev is not None:
                 ev[l][1].record(stream)
 
-    def timed(mode, K, per_kernel=False):
+    def capture(mode):
+        """The L-layer step as one CUDA graph (launch overhead leaves the timed loop)."""
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step(mode)  # warm the library's per-device caches outside capture
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=side):
+                step(mode)
+        torch.cuda.synchronize()
+        return g
+
+    def timed_graph(g, K):
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(K):
+            g.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return t0.elapsed_time(t1)
+
+    def timed_eager(mode, K):
         evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
-               for _ in range(K)] if per_kernel else None
+               for _ in range(K)]
         barrier()
         torch.cuda.synchronize()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for k in range(K):
-            step(mode, evs[k] if per_kernel else None)
+            step(mode, evs[k])
         t1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        total_ms = t0.elapsed_time(t1)
-        kern_ms = None
-        if per_kernel:
-            kern_ms = statistics.mean(e[0].elapsed_time(e[1]) for row in evs for e in row)
-        return total_ms, kern_ms
+        per = statistics.mean(e[0].elapsed_time(e[1]) for row in evs for e in row)
+        return t0.elapsed_time(t1), per
 
     for _ in range(args.warmup):
         step()
@@ -258,25 +281,33 @@ def main():
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} after warm-up")
 
+    graph = capture(W.GATE_TOPK)
+    for _ in range(args.warmup):
+        graph.replay()
     clocks = ClockSampler(local)
     clocks.start()
-    total_ms, kern_ms = timed(W.GATE_TOPK, args.steps, per_kernel=True)
+    total_ms = timed_graph(graph, args.steps)
     clk = clocks.stop()
     total_ms = max_over_ranks(total_ms)
-    kern_ms = max_over_ranks(kern_ms)
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
+    eager_ms, eager_kern_ms = timed_eager(W.GATE_TOPK, max(3, args.steps // 2))
+    eager_ms = max_over_ranks(eager_ms)
+    eager_kern_ms = max_over_ranks(eager_kern_ms)
 
     ms_per_step = total_ms / args.steps
     us_layer = ms_per_step * 1e3 / L
+    kern_ms = ms_per_step / L  # graph replay: per-launch time including the gap to the next launch
     gbs = world * nbytes * L * args.steps / (total_ms * 1e-3) / 1e9
 
     # dense comparator: the same kernel with every channel kept
+    dgraph = capture(W.GATE_DENSE)
     for _ in range(3):
-        step(W.GATE_DENSE)
-    dense_ms, _ = timed(W.GATE_DENSE, max(3, args.steps // 2))
-    dense_ms = max_over_ranks(dense_ms)
-    us_layer_dense = dense_ms / max(3, args.steps // 2) * 1e3 / L
+        dgraph.replay()
+    nd = max(3, args.steps // 2)
+    dense_ms = max_over_ranks(timed_graph(dgraph, nd))
+    us_layer_dense = dense_ms / nd * 1e3 / L
+    del dgraph
 
     # end to end through the C ABI: host x in pinned memory -> device, the call, y -> host
     hx = [x.cpu().pin_memory() for x in xs]
@@ -323,7 +354,9 @@ def main():
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
                      "kernel": "k_ffn_fused (one launch per layer)", "bytes_per_launch": nbytes,
-                     "kernel_us": kern_ms * 1e3},
+                     "kernel_us": kern_ms * 1e3, "timing": "CUDA graph of the L-layer step, events around K replays"},
+        "eager": {"us_per_layer": eager_ms / max(3, args.steps // 2) * 1e3 / L,
+                  "kernel_us_events": eager_kern_ms * 1e3},
         "dense": {"us_per_layer": us_layer_dense, "speedup": us_layer_dense / us_layer},
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "us_per_layer": e2e_ms / args.steps * 1e3 / L,
                 "h2d_bytes_per_step": L * D * 2, "d2h_bytes_per_step": L * D * 4},

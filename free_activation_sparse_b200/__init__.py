@@ -48,7 +48,8 @@ class _FfnT(ctypes.Structure):
 
 class _FfnView(ctypes.Structure):
     _fields_ = [("h", ctypes.c_size_t), ("idx_gate", ctypes.c_size_t), ("idx_up", ctypes.c_size_t),
-                ("idx_down", ctypes.c_size_t), ("cnt", ctypes.c_size_t)]
+                ("idx_down", ctypes.c_size_t), ("cnt", ctypes.c_size_t), ("stamps", ctypes.c_size_t),
+                ("cta_t", ctypes.c_size_t)]
 
 
 def _load() -> ctypes.CDLL:
@@ -266,8 +267,13 @@ class FfnWeights:
         return int(self.wt_gate.shape[1])
 
     def _struct(self) -> _FfnT:
-        return _FfnT(self.wt_gate.data_ptr(), self.wt_up.data_ptr(), self.wt_down.data_ptr(), _dt(self.wt_gate),
-                     self.c_gate.data_ptr(), self.c_up.data_ptr(), self.c_down.data_ptr(), self.d, self.ffn)
+        key = (self.wt_gate.data_ptr(), self.wt_up.data_ptr(), self.wt_down.data_ptr(), self.c_gate.data_ptr(),
+               self.c_up.data_ptr(), self.c_down.data_ptr())
+        cached = self.__dict__.get("_cstruct")
+        if cached is None or cached[0] != key:
+            st = _FfnT(key[0], key[1], key[2], _dt(self.wt_gate), key[3], key[4], key[5], self.d, self.ffn)
+            self.__dict__["_cstruct"] = cached = (key, st)
+        return cached[1]
 
 
 def ffn_prepare(W_gate, W_up, W_down) -> FfnWeights:
@@ -288,8 +294,7 @@ def sparse_ffn_swiglu(f: FfnWeights, x, mode: int = GATE_TOPK, k_gate: int = 0, 
         ws = Workspace(OP_FFN_SWIGLU, f.d, f.ffn, 0, B, device=x.device)
     if y is None:
         y = torch.empty((B, f.d), dtype=torch.float32, device=x.device)
-    fs = f._struct()
-    _check(lib.sparse_ffn_swiglu(ctypes.byref(fs), _ptr(x2), _dt(x2), B, int(mode), int(k_gate), int(k_up),
+    _check(lib.sparse_ffn_swiglu(ctypes.byref(f._struct()), _ptr(x2), _dt(x2), B, int(mode), int(k_gate), int(k_up),
                                  int(k_down), float(s), _ptr(y), ws.ptr, ws.nbytes, _ptr(status), _stream()),
            "sparse_ffn_swiglu")
     return y
@@ -297,14 +302,15 @@ def sparse_ffn_swiglu(f: FfnWeights, x, mode: int = GATE_TOPK, k_gate: int = 0, 
 
 def ffn_ws_view(ws: Workspace, d: int, ffn: int, batch: int) -> dict:
     """Views of the intermediate results a sparse_ffn_swiglu call leaves in `ws`:
-    h [B][ffn], idx_gate [B][d], idx_up [B][d], idx_down [B][ffn], cnt [3][B]."""
+    h [B][ffn], idx_gate [B][d], idx_up [B][d], idx_down [B][ffn], cnt [3][B], and the
+    single-token kernel's phase clock stamps [16] (int64 SM cycles of CTA 0)."""
     torch = _torch()
     v = _FfnView()
     _check(lib.wina_ffn_ws_view(d, ffn, batch, ctypes.byref(v)), "wina_ffn_ws_view")
     buf = ws.buf
 
     def take(off, count, dtype, shape):
-        nb = count * 4
+        nb = count * torch.empty(0, dtype=dtype).element_size()
         return buf[off: off + nb].view(dtype).view(*shape)
 
     return dict(
@@ -313,4 +319,6 @@ def ffn_ws_view(ws: Workspace, d: int, ffn: int, batch: int) -> dict:
         idx_up=take(v.idx_up, batch * d, torch.int32, (batch, d)),
         idx_down=take(v.idx_down, batch * ffn, torch.int32, (batch, ffn)),
         cnt=take(v.cnt, 3 * batch, torch.int32, (3, batch)),
+        stamps=take(v.stamps, 16, torch.int64, (16,)),
+        cta_t=take(v.cta_t, 296 * 4, torch.int64, (296, 4)),
     )

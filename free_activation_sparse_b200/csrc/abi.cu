@@ -2,15 +2,89 @@
 // used by the Spark threshold, workspace sizes and workspace views.
 #include <math.h>
 
+#include <mutex>
+
 #include "internal.h"
 
 namespace wina {
 
+// Small per-process caches of device facts, so that a launch does not query the
+// driver each time (the decode path is launch-latency sensitive).
+namespace {
+constexpr int kMaxDev = 64;
+constexpr int kCacheSlots = 128;
+struct OccEntry {
+  int dev;
+  const void* kern;
+  int threads;
+  size_t smem;
+  int per_sm;
+};
+struct SmemEntry {
+  int dev;
+  const void* kern;
+  size_t smem;
+};
+std::mutex g_mu;
+int g_sms[kMaxDev] = {0};
+OccEntry g_occ[kCacheSlots];
+int g_nocc = 0;
+SmemEntry g_smem[kCacheSlots];
+int g_nsmem = 0;
+}  // namespace
+
 int device_sm_count() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < kMaxDev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_sms[dev] > 0) return g_sms[dev];
+  }
+  int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < kMaxDev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_sms[dev] = sms;
+  }
   return sms;
+}
+
+cudaError_t ensure_smem_limit(const void* kern, size_t smem) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (int i = 0; i < g_nsmem; ++i)
+      if (g_smem[i].dev == dev && g_smem[i].kern == kern && g_smem[i].smem >= smem) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int i = 0; i < g_nsmem; ++i)
+    if (g_smem[i].dev == dev && g_smem[i].kern == kern) {
+      if (g_smem[i].smem < smem) g_smem[i].smem = smem;
+      return cudaSuccess;
+    }
+  if (g_nsmem < kCacheSlots) g_smem[g_nsmem++] = SmemEntry{dev, kern, smem};
+  return cudaSuccess;
+}
+
+int blocks_per_sm(const void* kern, int threads, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (int i = 0; i < g_nocc; ++i)
+      if (g_occ[i].dev == dev && g_occ[i].kern == kern && g_occ[i].threads == threads && g_occ[i].smem == smem)
+        return g_occ[i].per_sm;
+  }
+  if (smem > 48 * 1024 && ensure_smem_limit(kern, smem) != cudaSuccess) return 0;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_nocc < kCacheSlots) g_occ[g_nocc++] = OccEntry{dev, kern, threads, smem, per_sm};
+  return per_sm;
 }
 
 // Phi(z) = P(Z <= z) for a standard normal Z, via the complementary error function.
@@ -79,5 +153,7 @@ extern "C" wina_status_t wina_ffn_ws_view(int64_t d, int64_t ffn, int64_t batch,
   out->idx_up = L.idx_up;
   out->idx_down = L.idx_down;
   out->cnt = L.cnt;
+  out->stamps = L.stamps;
+  out->cta_t = L.cta_t;
   return WINA_OK;
 }

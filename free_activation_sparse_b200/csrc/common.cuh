@@ -111,64 +111,134 @@ struct Selection {
   uint32_t mask, prefix, r;
 };
 
-// Radix select of the K-th largest key (1 <= K < n) over keys[0..n) in SMEM, three
-// digit passes of 12, 12 and 8 bits from the top. After each pass the digit holding
-// the K-th key is fixed; if that digit's bin holds exactly the still-needed count, all
-// of it is kept and the search stops early. `hist` is SMEM of 4096 words, `red` SMEM of
-// >= 32 words. Every thread of the block must call it.
-template <int NT>
-__device__ Selection radix_select_topk(const uint32_t* keys, int n, int K, uint32_t* hist, uint32_t* red) {
-  __shared__ uint32_t s_digit, s_rem, s_cnt;
-  uint32_t mask = 0, prefix = 0, rem = (uint32_t)K;
+// Radix select of the K-th largest key over NSEL key arrays at once (each of length
+// n in SMEM, with its own K in [1, n)). Digits of 8, 8, 8 and 7 bits are taken from
+// bit 30 down (bit 31 of a non-negative float is 0). A pass histograms the digit of the
+// keys that still match the fixed prefix (SMEM atomics; two histogram buffers, the next
+// one cleared during the current pass), then warp q scans array q's 256 bins from the
+// top (8 per lane, one shuffle scan) and fixes the digit holding the K-th key. Two
+// block barriers per pass. A search ends early once that bin holds exactly the count
+// still needed. `hist` is SMEM of 2 * NSEL * 256 words; NSEL <= NT / 32. Every thread
+// of the block must call it.
+template <int NT, int NSEL>
+__device__ void radix_select(const uint32_t* const (&keys)[NSEL], int n, const int (&K)[NSEL], uint32_t* hist,
+                             Selection (&out)[NSEL]) {
+  __shared__ uint32_t s_res[NSEL][3];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t mask[NSEL], prefix[NSEL], rem[NSEL];
+  bool done[NSEL];
+#pragma unroll
+  for (int q = 0; q < NSEL; ++q) {
+    mask[q] = 0u;
+    prefix[q] = 0u;
+    rem[q] = (uint32_t)K[q];
+    done[q] = false;
+  }
+  for (int i = threadIdx.x; i < NSEL * 256; i += NT) hist[i] = 0u;
+  __syncthreads();
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int sh = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
-    const int nb = pass == 2 ? 256 : 4096;
-    const uint32_t dm = (uint32_t)nb - 1u;
-    for (int i = threadIdx.x; i < nb; i += NT) hist[i] = 0u;
-    __syncthreads();
+  for (int pass = 0; pass < 4; ++pass) {
+    const int sh = pass < 3 ? 23 - 8 * pass : 0;
+    const uint32_t dm = pass < 3 ? 0xffu : 0x7fu;
+    uint32_t* H = hist + (pass & 1) * NSEL * 256;
+    uint32_t* Hn = hist + ((pass & 1) ^ 1) * NSEL * 256;
     for (int i = threadIdx.x; i < n; i += NT) {
-      const uint32_t k = keys[i];
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> sh) & dm], 1u);
+#pragma unroll
+      for (int q = 0; q < NSEL; ++q) {
+        if (done[q]) continue;  // uniform across the block
+        const uint32_t k = keys[q][i];
+        if ((k & mask[q]) == prefix[q]) atomicAdd(&H[q * 256 + ((k >> sh) & dm)], 1u);
+      }
     }
+    for (int i = threadIdx.x; i < NSEL * 256; i += NT) Hn[i] = 0u;
     __syncthreads();
-    // Thread t owns the bins of descending rank [t*per, (t+1)*per): bin nb-1-q for q.
-    const int per = (nb + NT - 1) / NT;
-    const int q0 = threadIdx.x * per;
-    const int q1 = min(q0 + per, nb);
-    uint32_t local = 0;
-    for (int q = q0; q < q1; ++q) local += hist[nb - 1 - q];
-    const uint32_t above = block_excl_scan<NT>(local, red, nullptr);
-    if (above < rem && above + local >= rem) {  // exactly one thread holds the crossing
-      uint32_t cum = above;
-      for (int q = q0; q < q1; ++q) {
-        const uint32_t c = hist[nb - 1 - q];
-        if (cum + c >= rem) {
-          s_digit = (uint32_t)(nb - 1 - q);
-          s_rem = rem - cum;
-          s_cnt = c;
-          break;
+    if (warp < NSEL) {
+      const int q = warp;
+      if (!done[q]) {
+        uint32_t c[8];
+        uint32_t local = 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          c[j] = H[q * 256 + 255 - (lane * 8 + j)];  // descending bins
+          local += c[j];
         }
-        cum += c;
+        uint32_t incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const uint32_t above = incl - local;
+        if (above < rem[q] && incl >= rem[q]) {  // exactly one lane holds the crossing
+          uint32_t cum = above;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (cum + c[j] >= rem[q]) {
+              s_res[q][0] = 255u - (uint32_t)(lane * 8 + j);
+              s_res[q][1] = rem[q] - cum;
+              s_res[q][2] = c[j];
+              break;
+            }
+            cum += c[j];
+          }
+        }
       }
     }
     __syncthreads();
-    const uint32_t d = s_digit, cnt = s_cnt;
-    rem = s_rem;
-    prefix |= d << sh;
-    mask |= dm << sh;
-    __syncthreads();  // s_* and hist are rewritten by the next pass
-    if (cnt == rem) break;
+    bool all_done = true;
+#pragma unroll
+    for (int q = 0; q < NSEL; ++q) {
+      if (done[q]) continue;
+      rem[q] = s_res[q][1];
+      prefix[q] |= s_res[q][0] << sh;
+      mask[q] |= dm << sh;
+      if (s_res[q][2] == rem[q] || pass == 3) done[q] = true;
+      all_done = all_done && done[q];
+    }
+    if (all_done) break;
+    // s_res is rewritten only after the next pass's first barrier; H (this pass's
+    // buffer) is cleared by the next pass before its barrier, after everyone has
+    // passed the barrier above that ended the reads of it.
   }
-  return Selection{mask, prefix, rem};
+#pragma unroll
+  for (int q = 0; q < NSEL; ++q) out[q] = Selection{mask[q], prefix[q], rem[q]};
+  __syncthreads();
+}
+
+// Top-K of NSEL key arrays of length n (K = 0 and K >= n handled without a search).
+// `hist`: SMEM of 2 * NSEL * 256 words.
+template <int NT, int NSEL>
+__device__ __forceinline__ void select_topk_multi(const uint32_t* const (&keys)[NSEL], int n, const int (&K)[NSEL],
+                                                  uint32_t* hist, Selection (&out)[NSEL]) {
+  int Ks[NSEL];
+  bool search = false;
+#pragma unroll
+  for (int q = 0; q < NSEL; ++q) {
+    Ks[q] = K[q] <= 0 ? 0 : (K[q] >= n ? n : K[q]);
+    search = search || (Ks[q] > 0 && Ks[q] < n);
+  }
+  if (search) {
+    // arrays that need no search still run through the passes with K = 1 and are
+    // overwritten below; this keeps the block's control flow uniform
+    int Kr[NSEL];
+#pragma unroll
+    for (int q = 0; q < NSEL; ++q) Kr[q] = (Ks[q] > 0 && Ks[q] < n) ? Ks[q] : 1;
+    radix_select<NT, NSEL>(keys, n, Kr, hist, out);
+  }
+#pragma unroll
+  for (int q = 0; q < NSEL; ++q) {
+    if (Ks[q] == 0) out[q] = Selection{0u, 0u, 0u};
+    if (Ks[q] == n) out[q] = Selection{0u, 0u, (uint32_t)n};
+  }
 }
 
 template <int NT>
-__device__ __forceinline__ Selection select_topk_block(const uint32_t* keys, int n, int K, uint32_t* hist,
-                                                       uint32_t* red) {
-  if (K <= 0) return Selection{0u, 0u, 0u};
-  if (K >= n) return Selection{0u, 0u, (uint32_t)n};
-  return radix_select_topk<NT>(keys, n, K, hist, red);
+__device__ __forceinline__ Selection select_topk_block(const uint32_t* keys, int n, int K, uint32_t* hist) {
+  const uint32_t* ks[1] = {keys};
+  const int kk[1] = {K};
+  Selection out[1];
+  select_topk_multi<NT, 1>(ks, n, kk, hist, out);
+  return out[0];
 }
 
 // Warp-ballot compaction of a Selection, in ascending index order. Warp w walks the
@@ -327,20 +397,32 @@ __device__ Moments block_moments(Moments m, double* red) {
 }
 
 // ------------------------------------------------------------------------------------
-// grid barrier (cooperative launches only: all CTAs must be co-resident)
+// grid barriers (cooperative launches only: all CTAs must be co-resident)
 // ------------------------------------------------------------------------------------
 
-// Lives in the caller's workspace; zero-filled before first use. `count` returns to 0
-// after every completed barrier, `gen` only grows, so the state carries over between
-// calls without a reset.
+// Lives in the caller's workspace; zero-filled before first use.
 struct GridBarrier {
-  unsigned count;
-  unsigned gen;
-  unsigned pad[30];
+  unsigned count;            // grid_sync: arrivals of the current barrier (back to 0 after each)
+  unsigned gen;              // grid_sync: completed barriers
+  unsigned long long total;  // grid_sync_fixed: arrivals ever made
+  unsigned pad[28];
 };
 
-// Returns false if this CTA gave up waiting (WINA_ERR_TIMEOUT is recorded); the
-// caller must then return without touching shared results.
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long atom_add_release_u64(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.add.release.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
+// Sense-counting barrier that works for any grid size: the last arriver resets `count`
+// and bumps `gen`. Returns false if this CTA gave up waiting (WINA_ERR_TIMEOUT is
+// recorded); the caller must then return without touching shared results.
 __device__ __forceinline__ bool grid_sync(GridBarrier* bar, unsigned nblocks, int32_t* status) {
   __shared__ int s_ok;
   __syncthreads();
@@ -365,6 +447,34 @@ __device__ __forceinline__ bool grid_sync(GridBarrier* bar, unsigned nblocks, in
       }
     }
     __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// Barrier for kernels whose grid size never changes for a given workspace: arrivals
+// accumulate in a 64-bit counter, so barrier k of the workspace's life completes when
+// the counter reaches (k + 1) * nblocks. One release atomic per CTA and acquire polls;
+// the last arriver does no extra round trip. Same failure contract as grid_sync.
+__device__ __forceinline__ bool grid_sync_fixed(GridBarrier* bar, unsigned nblocks, int32_t* status) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const unsigned long long old = atom_add_release_u64(&bar->total, 1ull);
+    const unsigned long long target = old - old % nblocks + nblocks;
+    if (ld_acquire_u64(&bar->total) < target) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (ld_acquire_u64(&bar->total) < target) {
+        if (globaltimer_ns() - t0 > kBarrierTimeoutNs) {
+          ok = 0;
+          record_status(status, WINA_ERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(20);
+      }
+    }
     s_ok = ok;
   }
   __syncthreads();

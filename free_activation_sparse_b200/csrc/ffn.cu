@@ -25,7 +25,8 @@
 
 namespace wina {
 
-constexpr int kFfnRowCap = 512;  // kept rows one CTA stages per projection
+constexpr int kFfnRowCap = 512;             // kept rows one CTA stages per projection
+constexpr size_t kMaxSmem = 227 * 1024;     // dynamic SMEM one CTA may use on sm_100
 
 struct FfnParams {
   const void* wt_gate;
@@ -48,6 +49,8 @@ struct FfnParams {
   int32_t* idx_up;
   int32_t* idx_down;
   int32_t* cnt;
+  long long* stamps;
+  unsigned long long* cta_t;
   float* part_g;
   float* part_u;
   float* part_d;
@@ -105,42 +108,82 @@ __device__ void project(const void* __restrict__ Wt, const RowLayout& L, const i
   }
 }
 
-// For t < w: fixed-order sum over the CTAs pp that wrote a partial (wrote(pp)) of
-// part4[pp * m4 + c0 + t]. All threads must call it.
-template <typename Wrote>
-__device__ __forceinline__ float4 reduce_cols(const float4* __restrict__ part4, int64_t m4, int G, Wrote wrote,
-                                              int64_t c0, int w, float4* red4) {
+// Fixed-order column sums over the partial rows of the CTAs in `list` (nl entries,
+// ascending), for NP projections at once: for t < w, out[q] = sum over e of
+// part4[q][list[q][e] * m4 + c0 + t]. Thread (grp, ci) takes list entries grp,
+// grp + groups, ... and issues its loads eight at a time; the groups' sums are then
+// added in group order. `red4` is SMEM of NP * kNT float4. All threads must call it.
+template <int NP>
+__device__ __forceinline__ void reduce_lists(const float4* const (&part4)[NP], const int* const (&list)[NP],
+                                             const int (&nl)[NP], int64_t m4, int64_t c0, int w, float4* red4,
+                                             float4 (&out)[NP]) {
   const int groups = kNT / w;
   const int t = threadIdx.x;
   const int ci = t % w, grp = t / w;
-  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (grp < groups) {
-    for (int pp = grp; pp < G; pp += groups) {
-      if (!wrote(pp)) continue;
-      const float4 v = __ldcg(part4 + (int64_t)pp * m4 + c0 + ci);
-      a.x += v.x;
-      a.y += v.y;
-      a.z += v.z;
-      a.w += v.w;
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (grp < groups) {
+      const float4* base = part4[q] + c0 + ci;
+      const int* L = list[q];
+      for (int e0 = grp; e0 < nl[q]; e0 += 8 * groups) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {  // up to 8 independent loads in flight
+          const int e = e0 + u * groups;
+          v[u] = e < nl[q] ? __ldcg(base + (int64_t)L[e] * m4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          a.x += v[u].x;
+          a.y += v[u].y;
+          a.z += v[u].z;
+          a.w += v[u].w;
+        }
+      }
     }
+    red4[q * kNT + t] = a;
   }
-  red4[t] = a;
   __syncthreads();
-  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (t < w) {
-    for (int g = 0; g < groups; ++g) {
-      const float4 v = red4[g * w + t];
-      s.x += v.x;
-      s.y += v.y;
-      s.z += v.z;
-      s.w += v.w;
+#pragma unroll
+  for (int q = 0; q < NP; ++q) {
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < w) {
+      for (int g = 0; g < groups; ++g) {
+        const float4 v = red4[q * kNT + g * w + t];
+        s.x += v.x;
+        s.y += v.y;
+        s.z += v.z;
+        s.w += v.w;
+      }
     }
+    out[q] = s;
   }
   __syncthreads();
-  return s;
+}
+
+// Ascending list of the CTAs pp < G for which wrote(pp) holds; returns its length.
+template <typename Wrote>
+__device__ __forceinline__ int writer_list(int G, Wrote wrote, int* list, uint32_t* wsm) {
+  return (int)compact_pred<kNT>(
+      G, wrote,
+      [&](uint32_t total, uint32_t* lo, uint32_t* hi) {
+        *lo = 0;
+        *hi = total;
+      },
+      wsm, [&](int pp, uint32_t pos) { list[pos] = pp; });
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+// CTA 0 records its SM clock at phase boundaries; every CTA records the global timer at
+// the end of its four main phases (diagnostic views of the workspace).
+__device__ __forceinline__ void stamp(long long* stamps, int i) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) stamps[i] = clock64();
+}
+__device__ __forceinline__ void cta_time(unsigned long long* t, int i) {
+  if (threadIdx.x == 0) t[blockIdx.x * 4 + i] = globaltimer_ns();
+}
 
 template <bool BF16>
 __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
@@ -148,17 +191,20 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
   extern __shared__ __align__(16) unsigned char smraw[];
   const int d = a.d, ffn = a.ffn;
   const int nkeys = max(2 * d, ffn);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smraw);  // [nkeys]
-  uint32_t* hist = keys + nkeys;                         // [4096]
-  int32_t* rows = reinterpret_cast<int32_t*>(hist + 4096);  // [kFfnRowCap]
-  float* vals = reinterpret_cast<float*>(rows + kFfnRowCap);  // [kFfnRowCap]
-  float* red = vals + kFfnRowCap;                             // [kNT * 8]
-  float* fvals = reinterpret_cast<float*>(keys);
+  const int nvals = max(d, ffn);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smraw);          // [nkeys] scores (uint32 bits)
+  float* xv = reinterpret_cast<float*>(keys + nkeys);           // [nvals] x, then h
+  uint32_t* hist = reinterpret_cast<uint32_t*>(xv + nvals);     // [2 * 2 * 256] select histograms
+  int32_t* rows = reinterpret_cast<int32_t*>(hist + 1024);      // [kFfnRowCap]
+  float* vals = reinterpret_cast<float*>(rows + kFfnRowCap);    // [kFfnRowCap]
+  int* wl = reinterpret_cast<int*>(vals + kFfnRowCap);          // [2 * kGridCap] writer lists
+  float* red = reinterpret_cast<float*>(wl + 2 * kGridCap);     // [kNT * 8]
   __shared__ uint32_t wsm[2 * kNT / 32 + 1];
   __shared__ double dred[3 * kNT / 32];
 
   const int G = gridDim.x, b = blockIdx.x;
   const uint64_t pol = l2_evict_first_policy();
+  stamp(a.stamps, 0);
 
   // ---------------- A: gate / up selection ----------------
   int Kg, Ku;
@@ -167,7 +213,7 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
     Moments mo{0.0, 0.0, 0.0};
     for (int i = threadIdx.x; i < d; i += kNT) {
       const float f = load_elem(a.x, a.xdt, i);
-      fvals[i] = f;
+      xv[i] = f;
       mo.n += 1.0;
       const double dl = (double)f - mo.mean;
       mo.mean += dl / mo.n;
@@ -175,9 +221,9 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
     }
     const Moments tot = block_moments<kNT>(mo, dred);
     const double t = tot.mean + sqrt(tot.m2 / (double)d) * a.z;
-    auto pred = [&](int i) { return (double)fvals[i] > t; };
-    // gate part of the slice: the kept count is known only after the first walk;
-    // every thread computes the same split from it (no shared state needed)
+    auto pred = [&](int i) { return (double)xv[i] > t; };
+    // the kept count is known only after the first walk; every thread computes the
+    // same split from it (no shared state needed)
     int kept = 0;
     GateUpSplit gs{0, 0, 0, 0};
     compact_pred<kNT>(
@@ -191,7 +237,7 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
         wsm,
         [&](int i, uint32_t pos) {
           rows[pos - gs.g_lo] = i;
-          vals[pos - gs.g_lo] = fvals[i];
+          vals[pos - gs.g_lo] = xv[i];
           a.idx_gate[pos] = i;
         });
     Kg = Ku = kept;
@@ -206,75 +252,98 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
         wsm,
         [&](int i, uint32_t pos) {
           rows[ng + pos - sp.u_lo] = i;
-          vals[ng + pos - sp.u_lo] = fvals[i];
+          vals[ng + pos - sp.u_lo] = xv[i];
           a.idx_up[pos] = i;
         });
   } else {
-    Selection sg, su;
+    Selection sel[2];
     if (a.mode == WINA_GATE_TOPK) {
       for (int i = threadIdx.x; i < d; i += kNT) {
-        const float xv = load_elem(a.x, a.xdt, i);
-        keys[i] = __float_as_uint(fabsf(xv * __ldg(a.c_gate + i)));
-        keys[d + i] = __float_as_uint(fabsf(xv * __ldg(a.c_up + i)));
+        const float f = load_elem(a.x, a.xdt, i);
+        xv[i] = f;
+        keys[i] = __float_as_uint(fabsf(f * __ldg(a.c_gate + i)));
+        keys[d + i] = __float_as_uint(fabsf(f * __ldg(a.c_up + i)));
       }
       __syncthreads();
       Kg = a.k_gate;
       Ku = a.k_up;
-      sg = select_topk_block<kNT>(keys, d, Kg, hist, wsm);
-      su = select_topk_block<kNT>(keys + d, d, Ku, hist, wsm);
+      const uint32_t* ks[2] = {keys, keys + d};
+      const int kk[2] = {Kg, Ku};
+      select_topk_multi<kNT, 2>(ks, d, kk, hist, sel);
     } else {  // dense: every channel
-      for (int i = threadIdx.x; i < 2 * d; i += kNT) keys[i] = 0u;
+      for (int i = threadIdx.x; i < d; i += kNT) {
+        xv[i] = load_elem(a.x, a.xdt, i);
+        keys[i] = 0u;
+        keys[d + i] = 0u;
+      }
       __syncthreads();
       Kg = Ku = d;
-      sg = su = Selection{0u, 0u, (uint32_t)d};
+      sel[0] = sel[1] = Selection{0u, 0u, (uint32_t)d};
     }
     sp = gate_up_split(Kg, Ku, G, b);
     const int ng = sp.g_hi - sp.g_lo;
-    compact_selection<kNT>(keys, d, sg, (uint32_t)sp.g_lo, (uint32_t)sp.g_hi, wsm, [&](int i, uint32_t pos) {
+    compact_selection<kNT>(keys, d, sel[0], (uint32_t)sp.g_lo, (uint32_t)sp.g_hi, wsm, [&](int i, uint32_t pos) {
       rows[pos - sp.g_lo] = i;
-      vals[pos - sp.g_lo] = load_elem(a.x, a.xdt, i);
+      vals[pos - sp.g_lo] = xv[i];
       a.idx_gate[pos] = i;
     });
-    compact_selection<kNT>(keys + d, d, su, (uint32_t)sp.u_lo, (uint32_t)sp.u_hi, wsm, [&](int i, uint32_t pos) {
-      rows[ng + pos - sp.u_lo] = i;
-      vals[ng + pos - sp.u_lo] = load_elem(a.x, a.xdt, i);
-      a.idx_up[pos] = i;
-    });
+    compact_selection<kNT>(keys + d, d, sel[1], (uint32_t)sp.u_lo, (uint32_t)sp.u_hi, wsm,
+                           [&](int i, uint32_t pos) {
+                             rows[ng + pos - sp.u_lo] = i;
+                             vals[ng + pos - sp.u_lo] = xv[i];
+                             a.idx_up[pos] = i;
+                           });
   }
   __syncthreads();
+  stamp(a.stamps, 1);
+  cta_time(a.cta_t, 0);
 
   // ---------------- B: stream kept gate / up rows ----------------
   const RowLayout Lf = make_row_layout<kNT>(ffn, EPV);
   const int ng = sp.g_hi - sp.g_lo, nu = sp.u_hi - sp.u_lo;
   if (ng > 0) project<BF16>(a.wt_gate, Lf, rows, vals, ng, a.part_g + (int64_t)b * ffn, red, pol);
   if (nu > 0) project<BF16>(a.wt_up, Lf, rows + ng, vals + ng, nu, a.part_u + (int64_t)b * ffn, red, pol);
+  stamp(a.stamps, 2);
+  cta_time(a.cta_t, 1);
 
-  if (!grid_sync(a.bar, G, a.status)) return;
+  if (!grid_sync_fixed(a.bar, G, a.status)) return;
+  stamp(a.stamps, 3);
 
   // ---------------- C: g, u, h and the down scores for this CTA's columns ----------------
   {
+    int* lg = wl;
+    int* lu = wl + kGridCap;
+    const int ngl = writer_list(
+        G,
+        [&](int pp) {
+          const GateUpSplit s = gate_up_split(Kg, Ku, G, pp);
+          return s.g_hi > s.g_lo;
+        },
+        lg, wsm);
+    const int nul = writer_list(
+        G,
+        [&](int pp) {
+          const GateUpSplit s = gate_up_split(Kg, Ku, G, pp);
+          return s.u_hi > s.u_lo;
+        },
+        lu, wsm);
+    stamp(a.stamps, 10);
     const int64_t m4 = ffn / 4;
     const int64_t q0 = m4 * b / G, q1 = m4 * (b + 1) / G;
-    auto wrote_g = [&](int pp) {
-      const GateUpSplit s = gate_up_split(Kg, Ku, G, pp);
-      return s.g_hi > s.g_lo;
-    };
-    auto wrote_u = [&](int pp) {
-      const GateUpSplit s = gate_up_split(Kg, Ku, G, pp);
-      return s.u_hi > s.u_lo;
-    };
-    float4* red4 = reinterpret_cast<float4*>(red);
+    const float4* parts[2] = {reinterpret_cast<const float4*>(a.part_g), reinterpret_cast<const float4*>(a.part_u)};
+    const int* lists[2] = {lg, lu};
+    const int nls[2] = {ngl, nul};
     for (int64_t qb = q0; qb < q1; qb += kNT) {
       const int w = (int)min((int64_t)kNT, q1 - qb);
-      const float4 g4 = reduce_cols(reinterpret_cast<const float4*>(a.part_g), m4, G, wrote_g, qb, w, red4);
-      const float4 u4 = reduce_cols(reinterpret_cast<const float4*>(a.part_u), m4, G, wrote_u, qb, w, red4);
+      float4 gu[2];
+      reduce_lists<2>(parts, lists, nls, m4, qb, w, reinterpret_cast<float4*>(red), gu);
       if ((int)threadIdx.x < w) {
         const int64_t j = (qb + threadIdx.x) * 4;
         float4 h4;
-        h4.x = silu_f(g4.x) * u4.x;
-        h4.y = silu_f(g4.y) * u4.y;
-        h4.z = silu_f(g4.z) * u4.z;
-        h4.w = silu_f(g4.w) * u4.w;
+        h4.x = silu_f(gu[0].x) * gu[1].x;
+        h4.y = silu_f(gu[0].y) * gu[1].y;
+        h4.z = silu_f(gu[0].z) * gu[1].z;
+        h4.w = silu_f(gu[0].w) * gu[1].w;
         *reinterpret_cast<float4*>(a.h + j) = h4;
         if (a.mode == WINA_GATE_TOPK) {
           const float4 c4 = __ldg(reinterpret_cast<const float4*>(a.c_down + j));
@@ -289,27 +358,34 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
     }
   }
 
-  if (!grid_sync(a.bar, G, a.status)) return;
+  stamp(a.stamps, 4);
+  if (!grid_sync_fixed(a.bar, G, a.status)) return;
+  stamp(a.stamps, 5);
 
   // ---------------- D: down selection ----------------
   int Kd;
   Slice sd;
+  for (int i = threadIdx.x; i < ffn; i += kNT) {
+    xv[i] = __ldcg(a.h + i);
+    if (a.mode == WINA_GATE_TOPK) keys[i] = __ldcg(a.keys_d + i);
+  }
+  __syncthreads();
+  stamp(a.stamps, 11);
   if (a.mode == WINA_GATE_STAT) {
     Moments mo{0.0, 0.0, 0.0};
     for (int i = threadIdx.x; i < ffn; i += kNT) {
-      const float f = __ldcg(a.h + i);
-      fvals[i] = f;
+      const double f = (double)xv[i];
       mo.n += 1.0;
-      const double dl = (double)f - mo.mean;
+      const double dl = f - mo.mean;
       mo.mean += dl / mo.n;
-      mo.m2 += dl * ((double)f - mo.mean);
+      mo.m2 += dl * (f - mo.mean);
     }
     const Moments tot = block_moments<kNT>(mo, dred);
     const double t = tot.mean + sqrt(tot.m2 / (double)ffn) * a.z;
     int kept = 0;
     Slice ds{0, 0};
     compact_pred<kNT>(
-        ffn, [&](int i) { return (double)fvals[i] > t; },
+        ffn, [&](int i) { return (double)xv[i] > t; },
         [&](uint32_t total, uint32_t* lo, uint32_t* hi) {
           kept = (int)total;
           ds = slice_of(kept, G, b);
@@ -319,7 +395,7 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
         wsm,
         [&](int i, uint32_t pos) {
           rows[pos - ds.lo] = i;
-          vals[pos - ds.lo] = fvals[i];
+          vals[pos - ds.lo] = xv[i];
           a.idx_down[pos] = i;
         });
     Kd = kept;
@@ -327,10 +403,9 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
   } else {
     Selection sel;
     if (a.mode == WINA_GATE_TOPK) {
-      for (int i = threadIdx.x; i < ffn; i += kNT) keys[i] = __ldcg(a.keys_d + i);
-      __syncthreads();
       Kd = a.k_down;
-      sel = select_topk_block<kNT>(keys, ffn, Kd, hist, wsm);
+      sel = select_topk_block<kNT>(keys, ffn, Kd, hist);
+      stamp(a.stamps, 12);
     } else {
       Kd = ffn;
       sel = Selection{0u, 0u, (uint32_t)ffn};
@@ -338,7 +413,7 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
     sd = slice_of(Kd, G, b);
     compact_selection<kNT>(keys, ffn, sel, (uint32_t)sd.lo, (uint32_t)sd.hi, wsm, [&](int i, uint32_t pos) {
       rows[pos - sd.lo] = i;
-      vals[pos - sd.lo] = __ldcg(a.h + i);
+      vals[pos - sd.lo] = xv[i];
       a.idx_down[pos] = i;
     });
   }
@@ -348,34 +423,49 @@ __global__ void __launch_bounds__(kNT, 1) k_ffn_fused(FfnParams a) {
     a.cnt[1] = Ku;
     a.cnt[2] = Kd;
   }
+  stamp(a.stamps, 6);
+  cta_time(a.cta_t, 2);
 
   // ---------------- E: stream kept down rows ----------------
   const RowLayout Ld = make_row_layout<kNT>(d, EPV);
   const int nd = sd.hi - sd.lo;
   if (nd > 0) project<BF16>(a.wt_down, Ld, rows, vals, nd, a.part_d + (int64_t)b * d, red, pol);
+  stamp(a.stamps, 7);
+  cta_time(a.cta_t, 3);
 
-  if (!grid_sync(a.bar, G, a.status)) return;
+  if (!grid_sync_fixed(a.bar, G, a.status)) return;
+  stamp(a.stamps, 8);
 
   // ---------------- F: y for this CTA's columns ----------------
   {
+    int* ld = wl;
+    const int ndl = writer_list(
+        G,
+        [&](int pp) {
+          const Slice s = slice_of(Kd, G, pp);
+          return s.hi > s.lo;
+        },
+        ld, wsm);
     const int64_t m4 = d / 4;
     const int64_t q0 = m4 * b / G, q1 = m4 * (b + 1) / G;
-    auto wrote_d = [&](int pp) {
-      const Slice s = slice_of(Kd, G, pp);
-      return s.hi > s.lo;
-    };
-    float4* red4 = reinterpret_cast<float4*>(red);
+    const float4* parts[1] = {reinterpret_cast<const float4*>(a.part_d)};
+    const int* lists[1] = {ld};
+    const int nls[1] = {ndl};
     for (int64_t qb = q0; qb < q1; qb += kNT) {
       const int w = (int)min((int64_t)kNT, q1 - qb);
-      const float4 y4 = reduce_cols(reinterpret_cast<const float4*>(a.part_d), m4, G, wrote_d, qb, w, red4);
-      if ((int)threadIdx.x < w) reinterpret_cast<float4*>(a.y)[qb + threadIdx.x] = y4;
+      float4 y4[1];
+      reduce_lists<1>(parts, lists, nls, m4, qb, w, reinterpret_cast<float4*>(red), y4);
+      if ((int)threadIdx.x < w) reinterpret_cast<float4*>(a.y)[qb + threadIdx.x] = y4[0];
     }
   }
+  stamp(a.stamps, 9);
 }
 
 static size_t ffn_fused_smem(int64_t d, int64_t ffn) {
   const int64_t nkeys = 2 * d > ffn ? 2 * d : ffn;
-  return (size_t)nkeys * 4 + 4096 * 4 + (size_t)kFfnRowCap * 8 + (size_t)kNT * 8 * 4;
+  const int64_t nvals = d > ffn ? d : ffn;
+  return (size_t)nkeys * 4 + (size_t)nvals * 4 + (size_t)1024 * 4 + (size_t)kFfnRowCap * 8 +
+         (size_t)2 * kGridCap * 4 + (size_t)kNT * 8 * 4;
 }
 
 }  // namespace wina
@@ -415,7 +505,7 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
   const FfnWs L = ffn_ws_layout(d, ffn, batch);
   char* w = (char*)ws;
 
-  if (batch == 1 && 2 * d <= kMaxN) {
+  if (batch == 1 && 2 * d <= kMaxN && ffn_fused_smem(d, ffn) <= kMaxSmem) {
     const bool bf16 = f->wdt == WINA_BF16;
     const size_t smem = ffn_fused_smem(d, ffn);
     const int G = bf16 ? max_coresident_grid(k_ffn_fused<true>, kNT, smem)
@@ -446,6 +536,8 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
       p.idx_up = reinterpret_cast<int32_t*>(w + L.idx_up);
       p.idx_down = reinterpret_cast<int32_t*>(w + L.idx_down);
       p.cnt = reinterpret_cast<int32_t*>(w + L.cnt);
+      p.stamps = reinterpret_cast<long long*>(w + L.stamps);
+      p.cta_t = reinterpret_cast<unsigned long long*>(w + L.cta_t);
       p.part_g = reinterpret_cast<float*>(w + L.part_g);
       p.part_u = reinterpret_cast<float*>(w + L.part_u);
       p.part_d = reinterpret_cast<float*>(w + L.part_d);

@@ -16,6 +16,7 @@ constexpr int kGridCap = 296;
 constexpr int kNT = 512;          // threads per CTA of the selection / product kernels
 constexpr int kRowChunk = 1024;   // kept rows staged in SMEM at a time by sparse_matvec
 constexpr size_t kAlign = 256;    // alignment of every workspace sub-buffer
+constexpr int kFfnStamps = 16;    // phase clock stamps the single-token FFN kernel leaves
 
 inline bool valid_dtype(int dt) { return dt == WINA_F32 || dt == WINA_BF16; }
 inline int64_t elem_size(int dt) { return dt == WINA_BF16 ? 2 : 4; }
@@ -27,8 +28,16 @@ inline wina_status_t cuda_status(cudaError_t e) {
   return WINA_ERR_CUDA;
 }
 
-// Streaming multiprocessors of the current device (0 if none).
+// Streaming multiprocessors of the current device (0 if none). Cached per device.
 int device_sm_count();
+
+// Raise a kernel's dynamic SMEM limit to at least `smem` bytes on the current device
+// (remembered per device and kernel, so repeated calls cost a table lookup).
+cudaError_t ensure_smem_limit(const void* kern, size_t smem);
+
+// Co-resident CTAs per SM of `kern` at this block size and SMEM on the current device
+// (cached per device, kernel, block size and SMEM). 0 on error.
+int blocks_per_sm(const void* kern, int threads, size_t smem);
 
 // Launch with cudaLaunchKernelEx, optionally as a cooperative launch (all CTAs
 // co-resident, required by kernels that use grid_sync).
@@ -36,7 +45,7 @@ template <typename... Exp, typename... Act>
 cudaError_t launch_kernel(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool coop,
                           Act&&... args) {
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem_limit((const void*)kern, smem);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
@@ -57,12 +66,7 @@ cudaError_t launch_kernel(void (*kern)(Exp...), dim3 grid, dim3 block, size_t sm
 // Largest co-resident grid for `kern` at this block size and SMEM, capped at kGridCap.
 template <typename K>
 int max_coresident_grid(K kern, int threads, size_t smem) {
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return 0;
-  }
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess) return 0;
-  const int g = per_sm * device_sm_count();
+  const int g = blocks_per_sm((const void*)kern, threads, smem) * device_sm_count();
   return g < kGridCap ? g : kGridCap;
 }
 
@@ -86,11 +90,11 @@ inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
 
 // sparse_ffn_swiglu (d, ffn, batch):
 //   bar | h [B][ffn] | keys_d [B][ffn] | idx_gate [B][d] | idx_up [B][d] | idx_down [B][ffn]
-//   | cnt [3][B] | xs_gate [B][d] | xs_up [B][d] | xs_down [B][ffn] | g [B][ffn] | u [B][ffn]
+//   | cnt [3][B] | stamps [kFfnStamps] | cta_t [kGridCap][4] | xs_gate [B][d] | xs_up [B][d] | xs_down [B][ffn] | g [B][ffn] | u [B][ffn]
 //   | part_g [kGridCap][ffn] | part_u [kGridCap][ffn] | part_d [kGridCap][d] | spmv ws
 struct FfnWs {
-  size_t bar, h, keys_d, idx_gate, idx_up, idx_down, cnt, xs_gate, xs_up, xs_down, g, u, part_g, part_u, part_d,
-      spmv, total;
+  size_t bar, h, keys_d, idx_gate, idx_up, idx_down, cnt, stamps, cta_t, xs_gate, xs_up, xs_down, g, u, part_g,
+      part_u, part_d, spmv, total;
 };
 inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   FfnWs w;
@@ -107,6 +111,8 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   w.idx_up = take((size_t)B * d * 4);
   w.idx_down = take((size_t)B * ffn * 4);
   w.cnt = take((size_t)3 * B * 4);
+  w.stamps = take((size_t)kFfnStamps * 8);
+  w.cta_t = take((size_t)kGridCap * 4 * 8);
   w.xs_gate = take((size_t)B * d * 4);
   w.xs_up = take((size_t)B * d * 4);
   w.xs_down = take((size_t)B * ffn * 4);

@@ -2,7 +2,7 @@
 //
 //  * wina_select_topk ("WINA" article, section 一): score_i = |x_i * c_i| in float32,
 //    keep the K largest (ties to the lower index), written as an ascending index list.
-//    One CTA per token: scores live in SMEM as uint32 bit patterns, a three-pass radix
+//    One CTA per token: scores live in SMEM as uint32 bit patterns, a warp-ballot radix
 //    select finds the K-th largest, a two-walk warp-ballot compaction emits the list.
 //  * stat_topk_threshold ("Spark Transformer", section 2.2): mu, sigma^2 (divisor n) in
 //    one pass (Welford per thread, Chan's merge across threads, float64), then
@@ -19,7 +19,7 @@ __global__ void __launch_bounds__(NT) k_select_topk(const void* __restrict__ x, 
                                                     float* __restrict__ xs, float* __restrict__ scores) {
   extern __shared__ __align__(16) uint32_t sm[];
   uint32_t* keys = sm;       // [n]
-  uint32_t* hist = sm + n;   // [4096]
+  uint32_t* hist = sm + n;   // [512] select histograms
   __shared__ uint32_t red[64];
   const int64_t b = blockIdx.x;
   const int64_t off = b * (int64_t)n;
@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(NT) k_select_topk(const void* __restrict__ x, 
     if (scores) scores[off + i] = s;
   }
   __syncthreads();
-  const Selection sel = select_topk_block<NT>(keys, n, K, hist, red);
+  const Selection sel = select_topk_block<NT>(keys, n, K, hist);
   const int64_t ob = b * (int64_t)ld;
   compact_selection<NT>(keys, n, sel, 0u, (uint32_t)K, red, [&](int i, uint32_t pos) {
     idx[ob + pos] = i;
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(NT) k_stat_threshold(const void* __restrict__ 
 
 wina_status_t launch_select_topk(const void* x, int xdt, const float* c, int n, int k, int batch, int32_t* idx,
                                  float* xs, int ld, float* scores, cudaStream_t s) {
-  const size_t smem = (size_t)(n + 4096) * 4;
+  const size_t smem = (size_t)(n + 512) * 4;
   return cuda_status(launch_kernel(k_select_topk<kNT>, dim3(batch), dim3(kNT), smem, s, false, x, xdt, c, n, k, ld,
                                    idx, xs, scores));
 }

@@ -105,13 +105,23 @@ typedef struct {
  *   idx_gate int32  [batch][d]      kept gate channels, ascending (first cnt_gate[b])
  *   idx_up   int32  [batch][d]      kept up channels, ascending
  *   idx_down int32  [batch][ffn]    kept down channels, ascending
- *   cnt      int32  [3][batch]      kept counts of gate, up and down per token        */
+ *   cnt      int32  [3][batch]      kept counts of gate, up and down per token
+ *   stamps   int64  [16]            single-token kernel only: SM clock (clock64) of CTA 0
+ *                                   at its phase boundaries: 0 start, 1 gate/up selected,
+ *                                   2 gate/up rows streamed, 3 barrier, 4 h written,
+ *                                   5 barrier, 6 down selected, 7 down rows streamed,
+ *                                   8 barrier, 9 end
+ *   cta_t    uint64 [CTAs][4]       single-token kernel only: global timer (ns) at which
+ *                                   each CTA finished selecting gate/up, streaming
+ *                                   gate/up rows, selecting down, streaming down rows   */
 typedef struct {
   size_t h;
   size_t idx_gate;
   size_t idx_up;
   size_t idx_down;
   size_t cnt;
+  size_t stamps;
+  size_t cta_t;
 } wina_ffn_ws_view_t;
 
 /* ABI version of the loaded library (WINA_ABI_VERSION at build time). */
@@ -129,7 +139,8 @@ double wina_normal_quantile(double p);
 
 /* Bytes of device scratch that `op` needs for the given sizes (0 if none). The
  * workspace is owned by the caller, must be zero-filled before its first use, and may
- * be reused by later calls of the same op on the same stream; the library leaves it in
+ * be reused by later calls of the same op with the same sizes, on the same device and
+ * stream; the library leaves it in
  * a reusable state unless a call ended in WINA_ERR_TIMEOUT, after which it must be
  * zero-filled again. Concurrent calls need distinct workspaces.
  *   WINA_OP_SPARSE_MATVEC: n = in-features, m = out-features, k = max kept per token,

@@ -62,7 +62,8 @@ def test_ffn_ws_view_offsets_are_disjoint():
     v = W._FfnView()
     assert W.lib.wina_ffn_ws_view(4096, 11008, 2, ctypes.byref(v)) == W.OK
     spans = sorted([(v.h, 2 * 11008 * 4), (v.idx_gate, 2 * 4096 * 4), (v.idx_up, 2 * 4096 * 4),
-                    (v.idx_down, 2 * 11008 * 4), (v.cnt, 3 * 2 * 4)])
+                    (v.idx_down, 2 * 11008 * 4), (v.cnt, 3 * 2 * 4), (v.stamps, 16 * 8),
+                    (v.cta_t, 296 * 4 * 8)])
     for (a, la), (b, _) in zip(spans, spans[1:]):
         assert a + la <= b
         assert a % 256 == 0
