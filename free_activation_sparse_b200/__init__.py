@@ -5,7 +5,7 @@ of the computation runs in the library's CUDA kernels; this module only checks t
 dtypes/devices, allocates outputs and workspaces through PyTorch, passes raw device
 pointers and the current CUDA stream, and turns status codes into exceptions.
 Importing it fails if the library has not been built
-(``python -m free_activation_sparse_b200.build``).
+(``python free_activation_sparse_b200/build.py``).
 """
 
 from __future__ import annotations
@@ -18,7 +18,7 @@ __all__ = [
     "WinaError", "lib", "LIB_PATH", "F32", "BF16", "GATE_TOPK", "GATE_STAT", "GATE_DENSE",
     "abi_version", "normal_quantile", "workspace_size", "Workspace", "FfnWeights",
     "pack_in_major", "col_norms", "select_topk", "stat_topk_threshold", "sparse_matvec",
-    "sparse_ffn_swiglu", "ffn_ws_view", "ffn_prepare", "declared_symbols",
+    "sparse_ffn_swiglu", "ffn_ws_view", "ffn_prepare", "declared_symbols", "sparse_matvec_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwina.so")
@@ -54,7 +54,7 @@ class _FfnView(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m free_activation_sparse_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python free_activation_sparse_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     P, I64, I32, D, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double, ctypes.c_size_t
     E = ctypes.c_int
@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "wina_select_topk": (E, [P, E, P, I64, I64, I64, P, P, P, P]),
         "stat_topk_threshold": (E, [P, E, I64, D, I64, P, P, P, P, I64, P, P]),
         "sparse_matvec": (E, [P, E, I64, I64, P, P, I64, P, I64, I64, P, P, SZ, P, P]),
+        "sparse_matvec_noalloc": (E, [P, E, I64, I64, P, P, I64, P, I64, I64, P, P, P]),
         "sparse_ffn_swiglu": (E, [ctypes.POINTER(_FfnT), P, E, I64, E, I64, I64, I64, D, P, P, SZ, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -244,6 +245,29 @@ def sparse_matvec(Wt, idx, xs, k: int | None = None, count=None, ws: Workspace |
         y = torch.empty((B, m), dtype=torch.float32, device=Wt.device)
     _check(lib.sparse_matvec(_ptr(Wt), _dt(Wt), n, m, _ptr(idx2), _ptr(xs2), kk, _ptr(count), ld, B, _ptr(y),
                              ws.ptr, ws.nbytes, _ptr(status), _stream()), "sparse_matvec")
+    return y
+
+
+def sparse_matvec_noalloc(Wt, idx, xs, k: int | None = None, count=None, status=None, y=None):
+    """sparse_matvec without a workspace: the library's own fixed scratch is used (for
+    callers that cannot allocate device memory; see include/wina.h for its limit and
+    the rule that such calls must not overlap)."""
+    torch = _torch()
+    for t_, nm in ((Wt, "Wt"), (idx, "idx"), (xs, "xs"), (count, "count")):
+        _cuda(t_, nm)
+    if idx.dtype != torch.int32 or xs.dtype != torch.float32:
+        raise TypeError("idx must be int32 and xs float32")
+    idx2 = idx.reshape(1, -1) if idx.dim() == 1 else idx
+    xs2 = xs.reshape(1, -1) if xs.dim() == 1 else xs
+    n, m = Wt.shape
+    B, ld = idx2.shape
+    if k is None and count is None:
+        k = ld
+    kk = -1 if k is None else int(k)
+    if y is None:
+        y = torch.empty((B, m), dtype=torch.float32, device=Wt.device)
+    _check(lib.sparse_matvec_noalloc(_ptr(Wt), _dt(Wt), n, m, _ptr(idx2), _ptr(xs2), kk, _ptr(count), ld, B,
+                                     _ptr(y), _ptr(status), _stream()), "sparse_matvec_noalloc")
     return y
 
 

@@ -1,6 +1,8 @@
 """Build the CUDA library libwina.so in-tree (sm_100a, B200).
 
-    python -m free_activation_sparse_b200.build        # or build() from Python
+    python free_activation_sparse_b200/build.py [--force]   # or __graft_entry__.build()
+
+(Run it by path: importing the package loads libwina.so, which the build creates.)
 
 Compiles every csrc/*.cu with nvcc for sm_100a and links them into
 free_activation_sparse_b200/libwina.so (CUDA runtime linked statically), exporting

@@ -8,6 +8,8 @@
 // registers and writes one partial row. When P > 1 the launch is cooperative: after a
 // grid barrier (bounded wait) every CTA sums a slice of the outputs over the P partials
 // in a fixed order, so results are bit-reproducible. When P == 1 the CTA writes y.
+#include <mutex>
+
 #include "internal.h"
 
 namespace wina {
@@ -187,4 +189,93 @@ extern "C" wina_status_t sparse_matvec(const void* Wt, wina_dtype_t wdt, int64_t
   if (ws_bytes < wina_workspace_size(WINA_OP_SPARSE_MATVEC, n, m, ld_idx, batch)) return WINA_ERR_WORKSPACE;
   return launch_sparse_matvec(Wt, wdt, n, m, idx, xs, (int)k, count, (int)ld_idx, (int)batch, y, ws, status_dev,
                               (cudaStream_t)stream);
+}
+
+// ------------------------------------------------------------------------------------
+// sparse_matvec_noalloc: the same product with library-owned scratch
+// ------------------------------------------------------------------------------------
+//
+// Some callers cannot hand the library a workspace: code that runs where device
+// allocation is forbidden or too costly (a fixed memory pool owned by a host framework,
+// a latency-critical loop in which cudaMalloc could synchronise the device and stall
+// other streams, a plugin that only receives input and output buffers). For them this
+// entry point keeps its scratch (one grid-barrier word pair and the split-K partial
+// rows) in a fixed array in device memory that the library itself declares; every GPU
+// that loads the library holds it until the process exits.
+
+namespace wina {
+
+constexpr int64_t kNoAllocPartialFloats = (int64_t)1 << 21;  // 8 MiB of partial sums
+constexpr int64_t kNoAllocMaxOutputs = kNoAllocPartialFloats / 2;  // batch * m limit
+
+// [GridBarrier (256 B)][partials: kNoAllocPartialFloats float32]
+static __device__ __align__(256) unsigned char g_noalloc_scratch[256 + kNoAllocPartialFloats * 4];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {nullptr};
+}  // namespace
+
+// Device address of g_noalloc_scratch on the current device. In host code the array's
+// name is only a host-side stand-in, so the address is looked up once per device
+// (with that device current) and cached. Returns nullptr on error.
+static void* noalloc_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace wina
+
+extern "C" wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt, int64_t n, int64_t m,
+                                               const int32_t* idx, const float* xs, int64_t k, const int32_t* count,
+                                               int64_t ld_idx, int64_t batch, float* y, int32_t* status_dev,
+                                               wina_stream_t stream) {
+  if (!valid_dtype(wdt)) return WINA_ERR_UNSUPPORTED_DTYPE;
+  const int epv = wdt == WINA_BF16 ? 8 : 4;
+  if (n < 1 || n > INT32_MAX || m < epv || m % epv != 0 || m / epv > (int64_t)kNT * 8) return WINA_ERR_INVALID_ARG;
+  if (batch < 1 || batch > INT32_MAX || ld_idx < 0 || ld_idx > INT32_MAX) return WINA_ERR_INVALID_ARG;
+  if (batch * m > kNoAllocMaxOutputs) return WINA_ERR_INVALID_ARG;  // the fixed scratch is too small
+  if (k < -1 || k > ld_idx || (k == -1 && !count)) return WINA_ERR_INVALID_ARG;
+  if (!Wt || !y || (ld_idx > 0 && (!idx || !xs))) return WINA_ERR_INVALID_ARG;
+  if (!aligned(Wt, 16) || !aligned(y, 16) || (idx && !aligned(idx, 4)) || (xs && !aligned(xs, 4)) ||
+      (count && !aligned(count, 4)) || (status_dev && !aligned(status_dev, 4)))
+    return WINA_ERR_INVALID_ARG;
+  char* scratch = (char*)noalloc_scratch_ptr();
+  if (!scratch) return WINA_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  const bool bf16 = wdt == WINA_BF16;
+  const size_t smem = spmv_smem();
+  const int gmax = bf16 ? max_coresident_grid(k_sparse_matvec<true>, kNT, smem)
+                        : max_coresident_grid(k_sparse_matvec<false>, kNT, smem);
+  if (gmax < 1) return WINA_ERR_CUDA;
+  const int B = (int)batch;
+  int P = B < gmax ? gmax / B : 1;
+  const int kmax = k >= 0 ? (int)k : (int)ld_idx;
+  const int want = (kmax + 7) / 8;
+  if (P > want) P = want > 0 ? want : 1;
+  const int64_t fit = kNoAllocPartialFloats / (batch * m);  // partial rows per token that fit
+  if (P > fit) P = (int)fit;                                // >= 2 by the size check above
+  // The barrier words must start at zero: clear them on the stream (the partial rows
+  // are always written before they are read). Calls that overlap on the GPU share this
+  // scratch and race.
+  cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(GridBarrier), s);
+  if (e != cudaSuccess) return cuda_status(e);
+  GridBarrier* bar = reinterpret_cast<GridBarrier*>(scratch);
+  float* part = reinterpret_cast<float*>(scratch + 256);
+  const bool coop = P > 1;
+  const dim3 grid((unsigned)((int64_t)B * P));
+  if (bf16)
+    e = launch_kernel(k_sparse_matvec<true>, grid, dim3(kNT), smem, s, coop, Wt, n, m, idx, xs, (int)k, count,
+                      (int)ld_idx, P, y, part, bar, status_dev);
+  else
+    e = launch_kernel(k_sparse_matvec<false>, grid, dim3(kNT), smem, s, coop, Wt, n, m, idx, xs, (int)k, count,
+                      (int)ld_idx, P, y, part, bar, status_dev);
+  return cuda_status(e);
 }

@@ -220,6 +220,25 @@ wina_status_t sparse_matvec(const void* Wt, wina_dtype_t wdt, int64_t n, int64_t
                             const float* xs, int64_t k, const int32_t* count, int64_t ld_idx, int64_t batch,
                             float* y, void* ws, size_t ws_bytes, int32_t* status_dev, wina_stream_t stream);
 
+/* sparse_matvec for callers that cannot supply a workspace. The pages describe no
+ * such entry point; it exists for code that runs where device allocation is not an
+ * option (a framework that owns a fixed device memory pool, a latency-critical loop in
+ * which cudaMalloc could synchronise the device, a plugin that is only handed input and
+ * output buffers). Same arguments and results as sparse_matvec, minus ws / ws_bytes:
+ * the scratch (a barrier word pair and the split-K partial rows) lives in a fixed
+ * 8 MiB + 256 B array of device memory declared by the library, which every GPU that
+ * loads the library holds until the process exits. It allocates nothing.
+ *   Limit: batch * m <= 1,048,576 (at least two partial rows per token must fit in
+ *   the 2^21-float array); larger calls return WINA_ERR_INVALID_ARG.
+ *   The first call on a device looks up the array's device address (once per device,
+ *   with that device current); make that first call before any stream capture.
+ *   Every call clears the barrier words on `stream` and then reuses the same array:
+ *   calls that overlap on the GPU (other streams, other threads) race and must not
+ *   be issued. */
+wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt, int64_t n, int64_t m, const int32_t* idx,
+                                    const float* xs, int64_t k, const int32_t* count, int64_t ld_idx,
+                                    int64_t batch, float* y, int32_t* status_dev, wina_stream_t stream);
+
 /* SwiGLU FFN decode with the gate on every projection ("WAS" article: the gate is
  * applied per component, gate/up/down among them; "WINA" article, section 一: each
  * projection uses the column norms of its own weight and its own K):
