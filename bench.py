@@ -338,13 +338,13 @@ def main():
 
     peak, peak_kind = _peaks()
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
-    traffic = None
-    tf = os.path.join(ROOT, "profiles", "ffn_fused_llama7b_traffic.json")
+    traffic = None  # ncu dram bytes of one launch, valid only for the kernel it was taken on
+    tf = os.path.join(ROOT, "profiles", "ffn_fused_llama7b_traffic.txt")
     if os.path.exists(tf):
         with open(tf) as f:
-            tj = json.load(f)
-        if tj.get("p") == args.p and tj.get("kernel_sha") == _kernel_sha():
-            traffic = tj.get("dram_bytes_per_launch")
+            tj = dict(line.strip().split("=", 1) for line in f if "=" in line)
+        if float(tj.get("p", -1)) == args.p and tj.get("kernel_sha") == _kernel_sha():
+            traffic = int(tj["dram_bytes_per_launch"])
 
     line = {
         "metric": METRIC, "value": gbs, "unit": "GB/s", "us_per_layer": us_layer,

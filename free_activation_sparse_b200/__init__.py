@@ -47,9 +47,8 @@ class _FfnT(ctypes.Structure):
 
 
 class _FfnView(ctypes.Structure):
-    _fields_ = [("h", ctypes.c_size_t), ("idx_gate", ctypes.c_size_t), ("idx_up", ctypes.c_size_t),
-                ("idx_down", ctypes.c_size_t), ("cnt", ctypes.c_size_t), ("stamps", ctypes.c_size_t),
-                ("cta_t", ctypes.c_size_t)]
+    _fields_ = [("h", ctypes.c_size_t), ("keep_gate", ctypes.c_size_t), ("keep_up", ctypes.c_size_t),
+                ("keep_down", ctypes.c_size_t), ("stamps", ctypes.c_size_t), ("cta_t", ctypes.c_size_t)]
 
 
 def _load() -> ctypes.CDLL:
@@ -326,8 +325,9 @@ def sparse_ffn_swiglu(f: FfnWeights, x, mode: int = GATE_TOPK, k_gate: int = 0, 
 
 def ffn_ws_view(ws: Workspace, d: int, ffn: int, batch: int) -> dict:
     """Views of the intermediate results a sparse_ffn_swiglu call leaves in `ws`:
-    h [B][ffn], idx_gate [B][d], idx_up [B][d], idx_down [B][ffn], cnt [3][B], and the
-    single-token kernel's phase clock stamps [16] (int64 SM cycles of CTA 0)."""
+    h [B][ffn] float32; keep_gate, keep_up [B][d] and keep_down [B][ffn] as 0/1 bytes;
+    the single-token kernel's phase clock stamps [16] (int64 SM cycles of CTA 0) and
+    per-CTA phase end times cta_t [296][4] (int64 ns)."""
     torch = _torch()
     v = _FfnView()
     _check(lib.wina_ffn_ws_view(d, ffn, batch, ctypes.byref(v)), "wina_ffn_ws_view")
@@ -339,10 +339,9 @@ def ffn_ws_view(ws: Workspace, d: int, ffn: int, batch: int) -> dict:
 
     return dict(
         h=take(v.h, batch * ffn, torch.float32, (batch, ffn)),
-        idx_gate=take(v.idx_gate, batch * d, torch.int32, (batch, d)),
-        idx_up=take(v.idx_up, batch * d, torch.int32, (batch, d)),
-        idx_down=take(v.idx_down, batch * ffn, torch.int32, (batch, ffn)),
-        cnt=take(v.cnt, 3 * batch, torch.int32, (3, batch)),
+        keep_gate=take(v.keep_gate, batch * d, torch.uint8, (batch, d)),
+        keep_up=take(v.keep_up, batch * d, torch.uint8, (batch, d)),
+        keep_down=take(v.keep_down, batch * ffn, torch.uint8, (batch, ffn)),
         stamps=take(v.stamps, 16, torch.int64, (16,)),
         cta_t=take(v.cta_t, 296 * 4, torch.int64, (296, 4)),
     )

@@ -149,10 +149,9 @@ extern "C" wina_status_t wina_ffn_ws_view(int64_t d, int64_t ffn, int64_t batch,
   if (d < 1 || ffn < 1 || batch < 1 || !out) return WINA_ERR_INVALID_ARG;
   const FfnWs L = ffn_ws_layout(d, ffn, batch);
   out->h = L.h;
-  out->idx_gate = L.idx_gate;
-  out->idx_up = L.idx_up;
-  out->idx_down = L.idx_down;
-  out->cnt = L.cnt;
+  out->keep_gate = L.keep_g;
+  out->keep_up = L.keep_u;
+  out->keep_down = L.keep_d;
   out->stamps = L.stamps;
   out->cta_t = L.cta_t;
   return WINA_OK;

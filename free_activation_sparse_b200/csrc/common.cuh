@@ -106,9 +106,10 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* red, u
 // A selection over keys: channel i is kept iff
 //     (key_i & mask) >  prefix                                  (strictly above), or
 //     (key_i & mask) == prefix and its rank among such i < r      (boundary, by index).
-// K = n is {0, 0, n}; K = 0 is {0, 0, 0}.
+// neq counts the boundary channels; when r == neq every boundary channel is kept.
+// K = n is {0, 0, n, n}; K = 0 is {0, 0, 0, n}.
 struct Selection {
-  uint32_t mask, prefix, r;
+  uint32_t mask, prefix, r, neq;
 };
 
 // Radix select of the K-th largest key over NSEL key arrays at once (each of length
@@ -125,13 +126,14 @@ __device__ void radix_select(const uint32_t* const (&keys)[NSEL], int n, const i
                              Selection (&out)[NSEL]) {
   __shared__ uint32_t s_res[NSEL][3];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t mask[NSEL], prefix[NSEL], rem[NSEL];
+  uint32_t mask[NSEL], prefix[NSEL], rem[NSEL], neq[NSEL];
   bool done[NSEL];
 #pragma unroll
   for (int q = 0; q < NSEL; ++q) {
     mask[q] = 0u;
     prefix[q] = 0u;
     rem[q] = (uint32_t)K[q];
+    neq[q] = (uint32_t)n;
     done[q] = false;
   }
   for (int i = threadIdx.x; i < NSEL * 256; i += NT) hist[i] = 0u;
@@ -190,9 +192,10 @@ __device__ void radix_select(const uint32_t* const (&keys)[NSEL], int n, const i
     for (int q = 0; q < NSEL; ++q) {
       if (done[q]) continue;
       rem[q] = s_res[q][1];
+      neq[q] = s_res[q][2];
       prefix[q] |= s_res[q][0] << sh;
       mask[q] |= dm << sh;
-      if (s_res[q][2] == rem[q] || pass == 3) done[q] = true;
+      if (neq[q] == rem[q] || pass == 3) done[q] = true;
       all_done = all_done && done[q];
     }
     if (all_done) break;
@@ -201,7 +204,7 @@ __device__ void radix_select(const uint32_t* const (&keys)[NSEL], int n, const i
     // passed the barrier above that ended the reads of it.
   }
 #pragma unroll
-  for (int q = 0; q < NSEL; ++q) out[q] = Selection{mask[q], prefix[q], rem[q]};
+  for (int q = 0; q < NSEL; ++q) out[q] = Selection{mask[q], prefix[q], rem[q], neq[q]};
   __syncthreads();
 }
 
@@ -227,8 +230,8 @@ __device__ __forceinline__ void select_topk_multi(const uint32_t* const (&keys)[
   }
 #pragma unroll
   for (int q = 0; q < NSEL; ++q) {
-    if (Ks[q] == 0) out[q] = Selection{0u, 0u, 0u};
-    if (Ks[q] == n) out[q] = Selection{0u, 0u, (uint32_t)n};
+    if (Ks[q] == 0) out[q] = Selection{0u, 0u, 0u, (uint32_t)n};
+    if (Ks[q] == n) out[q] = Selection{0u, 0u, (uint32_t)n, (uint32_t)n};
   }
 }
 
@@ -352,6 +355,341 @@ __device__ uint32_t compact_pred(int n, Pred pred, Range range, uint32_t* wsm, E
   }
   __syncthreads();
   return total;
+}
+
+// ------------------------------------------------------------------------------------
+// top-K as a threshold: kept(j) <=> key_j > T, or key_j == T and j <= cut
+// ------------------------------------------------------------------------------------
+
+struct Threshold {
+  uint32_t T;  // key of the K-th largest channel
+  int cut;     // its index: among keys equal to T, those with index <= cut are kept
+};
+
+__device__ __forceinline__ bool kept_by(const Threshold& t, uint32_t key, int j) {
+  return key > t.T || (key == t.T && j <= t.cut);
+}
+
+constexpr int kSelBins = 4096;   // histogram bins of select_threshold
+constexpr int kSelCand = 512;    // candidates resolved exactly by ranking
+
+// Block-wide min and max of v (all threads receive them). `red` >= 2 * NT/32 words.
+template <int NT>
+__device__ __forceinline__ void block_minmax_u32(uint32_t v_min, uint32_t v_max, uint32_t* red, uint32_t& mn,
+                                                 uint32_t& mx) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v_min = __reduce_min_sync(0xffffffffu, v_min);
+  v_max = __reduce_max_sync(0xffffffffu, v_max);
+  if (lane == 0) {
+    red[warp] = v_min;
+    red[NW + warp] = v_max;
+  }
+  __syncthreads();
+  mn = 0xffffffffu;
+  mx = 0u;
+  for (int w = 0; w < NW; ++w) {
+    mn = min(mn, red[w]);
+    mx = max(mx, red[NW + w]);
+  }
+  __syncthreads();
+}
+
+// Exact top-K of keys[0..n) in SMEM (ties to the lower index), found as a threshold.
+// The candidates (initially every key) are spread over kSelBins bins by a linear map
+// of their bit patterns between the candidates' min and max key; the map is monotone,
+// so the bins are ordered like the keys. One histogram pass and a scan find the bin
+// holding the K-th key; if that bin holds at most kSelCand keys they are ranked
+// exactly, otherwise the search repeats inside the bin's key range. Equal keys are
+// ordered by index. Buffers in SMEM: hist [kSelBins], cand [2 * kSelCand] words,
+// red [>= 2 * NT/32 + 4] words. Every thread of the block must call it.
+template <int NT>
+__device__ Threshold select_threshold(const uint32_t* __restrict__ keys, int n, int K, uint32_t* __restrict__ hist,
+                                      uint32_t* __restrict__ cand, uint32_t* __restrict__ red) {
+  constexpr int CH = 8;  // keys a thread loads into registers before it updates counts
+  __shared__ uint32_t s_bin, s_above, s_cnt, s_ncand;
+  __shared__ Threshold s_res;
+  if (K <= 0) return Threshold{0xffffffffu, -1};
+  if (K >= n) return Threshold{0u, n - 1};
+  uint32_t lo = 0u, hi = 0xffffffffu;  // key range of the candidates
+  uint32_t r = (uint32_t)K;            // rank (1-based, from the top) sought among them
+#pragma unroll 1
+  for (int iter = 0; iter < 8; ++iter) {
+    // candidates' min / max
+    uint32_t a = 0xffffffffu, b = 0u;
+    for (int i0 = threadIdx.x; i0 < n; i0 += CH * NT) {
+      uint32_t k[CH];
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int i = i0 + u * NT;
+        k[u] = i < n ? keys[i] : lo;  // lo never widens [a, b] beyond the candidates
+      }
+#pragma unroll
+      for (int u = 0; u < CH; ++u)
+        if (k[u] >= lo && k[u] <= hi) {
+          a = min(a, k[u]);
+          b = max(b, k[u]);
+        }
+    }
+    uint32_t mn, mx;
+    block_minmax_u32<NT>(a, b, red, mn, mx);
+    if (mn == mx) {
+      // every candidate has the same key: the r-th of them by index is the cut
+      if (threadIdx.x == 0) s_res = Threshold{mn, n - 1};
+      compact_pred<NT>(
+          n, [&](int i) { return keys[i] == mn; },
+          [&](uint32_t, uint32_t* l, uint32_t* h) {
+            *l = r - 1;
+            *h = r;
+          },
+          red, [&](int i, uint32_t) { s_res.cut = i; });
+      const Threshold t = s_res;
+      __syncthreads();
+      return t;
+    }
+    const float scale = (float)kSelBins / ((float)(mx - mn) + 1.0f);
+    auto bin_of = [&](uint32_t k) { return min(kSelBins - 1, (int)((float)(k - mn) * scale)); };
+    for (int i = threadIdx.x; i < kSelBins; i += NT) hist[i] = 0u;
+    if (threadIdx.x == 0) s_ncand = 0u;
+    __syncthreads();
+    for (int i0 = threadIdx.x; i0 < n; i0 += CH * NT) {
+      uint32_t k[CH];
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int i = i0 + u * NT;
+        k[u] = i < n ? keys[i] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < CH; ++u)
+        if (i0 + u * NT < n && k[u] >= mn && k[u] <= mx) atomicAdd(&hist[bin_of(k[u])], 1u);
+    }
+    __syncthreads();
+    // bins from the top: thread t owns descending bins [t*per, (t+1)*per)
+    constexpr int per = (kSelBins + NT - 1) / NT;
+    const int q0 = threadIdx.x * per, q1 = min(q0 + per, kSelBins);
+    uint32_t local = 0u;
+    for (int q = q0; q < q1; ++q) local += hist[kSelBins - 1 - q];
+    const uint32_t above = block_excl_scan<NT>(local, red, nullptr);
+    if (above < r && above + local >= r) {  // exactly one thread holds the crossing
+      uint32_t cum = above;
+      for (int q = q0; q < q1; ++q) {
+        const uint32_t c = hist[kSelBins - 1 - q];
+        if (cum + c >= r) {
+          s_bin = (uint32_t)(kSelBins - 1 - q);
+          s_above = cum;
+          s_cnt = c;
+          break;
+        }
+        cum += c;
+      }
+    }
+    __syncthreads();
+    const int bin = (int)s_bin;
+    const uint32_t cnt = s_cnt;
+    r -= s_above;
+    if (cnt <= (uint32_t)kSelCand) {
+      // gather the bin's keys and rank them exactly: (key desc, index asc)
+      for (int i0 = threadIdx.x; i0 < n; i0 += CH * NT) {
+        uint32_t k[CH];
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+          const int i = i0 + u * NT;
+          k[u] = i < n ? keys[i] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+          const int i = i0 + u * NT;
+          if (i < n && k[u] >= mn && k[u] <= mx && bin_of(k[u]) == bin) {
+            const uint32_t at = atomicAdd(&s_ncand, 1u);
+            cand[2 * at] = k[u];
+            cand[2 * at + 1] = (uint32_t)i;
+          }
+        }
+      }
+      __syncthreads();
+      const int nc = (int)s_ncand;
+      for (int c = threadIdx.x; c < nc; c += NT) {
+        const uint32_t kc = cand[2 * c];
+        const int ic = (int)cand[2 * c + 1];
+        uint32_t rank = 0u;
+        for (int o = 0; o < nc; ++o) {
+          const uint32_t ko = cand[2 * o];
+          const int io = (int)cand[2 * o + 1];
+          rank += (ko > kc || (ko == kc && io < ic)) ? 1u : 0u;
+        }
+        if (rank == r - 1) s_res = Threshold{kc, ic};
+      }
+      __syncthreads();
+      const Threshold t = s_res;
+      __syncthreads();
+      return t;
+    }
+    // too many keys in the bin: narrow the range to the bin's members and repeat
+    uint32_t a2 = 0xffffffffu, b2 = 0u;
+    for (int i0 = threadIdx.x; i0 < n; i0 += CH * NT) {
+      uint32_t k[CH];
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int i = i0 + u * NT;
+        k[u] = i < n ? keys[i] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < CH; ++u)
+        if (i0 + u * NT < n && k[u] >= mn && k[u] <= mx && bin_of(k[u]) == bin) {
+          a2 = min(a2, k[u]);
+          b2 = max(b2, k[u]);
+        }
+    }
+    block_minmax_u32<NT>(a2, b2, red, lo, hi);
+  }
+  return Threshold{lo, n - 1};  // not reached for 32-bit keys (each round shrinks the range)
+}
+
+// Bin holding the r-th largest of kSelBins counts, scanned from the top in two levels:
+// warp w (< 16) sums its 256 contiguous bins with conflict-free loads, warp 0 scans
+// the 16 totals, and the warp whose chunk holds the crossing scans its 8 rows of 32
+// bins. Results in *bin (the bin), *above (count in higher bins), *cnt (the bin's
+// count). Requires NT >= 512. Every thread must call it.
+template <int NT>
+__device__ void hist_crossing(const uint32_t* __restrict__ hist, uint32_t r, uint32_t* red, int* bin,
+                              uint32_t* above, uint32_t* cnt) {
+  static_assert(NT >= 512, "needs 16 warps");
+  __shared__ uint32_t s_w, s_wabove, s_bin, s_above, s_cnt;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp < 16) {
+    const int top = kSelBins - 1 - warp * 256;  // the warp's bins top, top-1, ..., top-255
+    uint32_t t = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t += hist[top - (j * 32 + lane)];
+    t = __reduce_add_sync(0xffffffffu, t);
+    if (lane == 0) red[warp] = t;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t v = lane < 16 ? red[lane] : 0u;
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const bool hit = lane < 16 && inc - v < r && inc >= r;
+    const uint32_t m = __ballot_sync(0xffffffffu, hit);
+    const int w = __ffs(m) - 1;
+    if (lane == w) {
+      s_w = (uint32_t)w;
+      s_wabove = inc - v;
+    }
+  }
+  __syncthreads();
+  if (warp == (int)s_w) {
+    const int top = kSelBins - 1 - warp * 256;
+    uint32_t base = s_wabove;
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t v = hist[top - (j * 32 + lane)];
+      uint32_t inc = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const uint32_t ab = base + inc - v;
+      const uint32_t m = __ballot_sync(0xffffffffu, ab < r && ab + v >= r);
+      if (m) {
+        const int l = __ffs(m) - 1;
+        if (lane == l) {
+          s_bin = (uint32_t)(top - (j * 32 + l));
+          s_above = ab;
+          s_cnt = v;
+        }
+        break;
+      }
+      base = __shfl_sync(0xffffffffu, base + inc, 31);
+    }
+  }
+  __syncthreads();
+  *bin = (int)s_bin;
+  *above = s_above;
+  *cnt = s_cnt;
+}
+
+// Kept-channel bitmask of the exact top-K of keys[0..n) in SMEM (ties to the lower
+// index), given the keys' min and max. One histogram pass over a linear map of the key
+// bits onto kSelBins bins (monotone, so bins are ordered like the keys), a two-level
+// scan for the bin holding the K-th key, then one pass that sets the flags of every
+// channel outside that bin and gathers the bin's keys; those are ranked exactly and
+// the kept ones set. If the bin holds more than kSelCand keys, the general search
+// (select_threshold) decides. flags[w] bit l = channel 32w + l is kept.
+// SMEM: hist [kSelBins], cand [2 * kSelCand], red [>= 2 * NT/32 + 8]. All threads call.
+template <int NT>
+__device__ void select_topk_flags(const uint32_t* __restrict__ keys, int n, int K, uint32_t mn, uint32_t mx,
+                                  uint32_t* __restrict__ hist, uint32_t* __restrict__ cand, uint32_t* __restrict__ red,
+                                  uint32_t* __restrict__ flags) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = (n + 31) / 32;
+  __shared__ uint32_t s_ncand;
+  if (K <= 0 || K >= n || mn == mx) {
+    // nothing, everything, or all keys equal (then the first K by index)
+    const int keep = K <= 0 ? 0 : (K >= n ? n : K);
+    for (int w = threadIdx.x; w < nw; w += NT) {
+      const int rem = keep - w * 32;
+      flags[w] = rem >= 32 ? 0xffffffffu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
+    }
+    __syncthreads();
+    return;
+  }
+  const float scale = (float)kSelBins / ((float)(mx - mn) + 1.0f);
+  auto bin_of = [&](uint32_t k) { return min(kSelBins - 1, (int)((float)(k - mn) * scale)); };
+  for (int i = threadIdx.x; i < kSelBins; i += NT) hist[i] = 0u;
+  if (threadIdx.x == 0) s_ncand = 0u;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += NT) atomicAdd(&hist[bin_of(keys[i])], 1u);
+  __syncthreads();
+  int B;
+  uint32_t above, cnt;
+  hist_crossing<NT>(hist, (uint32_t)K, red, &B, &above, &cnt);
+  if (cnt > (uint32_t)kSelCand) {
+    const Threshold t = select_threshold<NT>(keys, n, K, hist, cand, red);
+    for (int w = warp; w < nw; w += NW) {
+      const int j = w * 32 + lane;
+      const uint32_t bits = __ballot_sync(0xffffffffu, j < n && kept_by(t, keys[j], j));
+      if (lane == 0) flags[w] = bits;
+    }
+    __syncthreads();
+    return;
+  }
+  const uint32_t r = (uint32_t)K - above;  // kept among the bin's keys
+  for (int w = warp; w < nw; w += NW) {
+    const int j = w * 32 + lane;
+    int bj = -1;
+    uint32_t k = 0u;
+    if (j < n) {
+      k = keys[j];
+      bj = bin_of(k);
+    }
+    const uint32_t bits = __ballot_sync(0xffffffffu, bj > B);
+    if (lane == 0) flags[w] = bits;
+    if (bj == B) {
+      const uint32_t at = atomicAdd(&s_ncand, 1u);
+      cand[2 * at] = k;
+      cand[2 * at + 1] = (uint32_t)j;
+    }
+  }
+  __syncthreads();
+  const int nc = (int)s_ncand;
+  for (int c = threadIdx.x; c < nc; c += NT) {
+    const uint32_t kc = cand[2 * c];
+    const int ic = (int)cand[2 * c + 1];
+    uint32_t rank = 0u;
+    for (int o = 0; o < nc; ++o) {
+      const uint32_t ko = cand[2 * o];
+      const int io = (int)cand[2 * o + 1];
+      rank += (ko > kc || (ko == kc && io < ic)) ? 1u : 0u;
+    }
+    if (rank < r) atomicOr(&flags[ic >> 5], 1u << (ic & 31));
+  }
+  __syncthreads();
 }
 
 // ------------------------------------------------------------------------------------

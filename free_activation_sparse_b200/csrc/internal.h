@@ -16,7 +16,7 @@ constexpr int kGridCap = 296;
 constexpr int kNT = 512;          // threads per CTA of the selection / product kernels
 constexpr int kRowChunk = 1024;   // kept rows staged in SMEM at a time by sparse_matvec
 constexpr size_t kAlign = 256;    // alignment of every workspace sub-buffer
-constexpr int kFfnStamps = 16;    // phase clock stamps the single-token FFN kernel leaves
+constexpr int kFfnStamps = 16 + 256;  // phase clock stamps + a stage trace the single-token FFN kernel leaves
 
 inline bool valid_dtype(int dt) { return dt == WINA_F32 || dt == WINA_BF16; }
 inline int64_t elem_size(int dt) { return dt == WINA_BF16 ? 2 : 4; }
@@ -89,12 +89,15 @@ inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
 }
 
 // sparse_ffn_swiglu (d, ffn, batch):
-//   bar | h [B][ffn] | keys_d [B][ffn] | idx_gate [B][d] | idx_up [B][d] | idx_down [B][ffn]
-//   | cnt [3][B] | stamps [kFfnStamps] | cta_t [kGridCap][4] | xs_gate [B][d] | xs_up [B][d] | xs_down [B][ffn] | g [B][ffn] | u [B][ffn]
-//   | part_g [kGridCap][ffn] | part_u [kGridCap][ffn] | part_d [kGridCap][d] | spmv ws
+//   bar | ctr [8] (unit counters, done, epoch) | h [B][ffn] | keep_g [B][d] | keep_u [B][d] (bytes)
+//   | keep_d [B][ffn] (bytes) | stamps [kFfnStamps] | cta_t [kGridCap][4]
+//   | idx_gate, idx_up [B][d] | idx_down [B][ffn] | cnt [3][B] | xs_gate, xs_up [B][d]
+//   | xs_down [B][ffn] | g, u [B][ffn]                       (several tokens)
+//   | acc_g, acc_u [2][ffn] | acc_y [d]                       (one token)
+//   | spmv ws                                                 (several tokens)
 struct FfnWs {
-  size_t bar, h, keys_d, idx_gate, idx_up, idx_down, cnt, stamps, cta_t, xs_gate, xs_up, xs_down, g, u, part_g,
-      part_u, part_d, spmv, total;
+  size_t bar, ctr, h, keep_g, keep_u, keep_d, stamps, cta_t, idx_gate, idx_up, idx_down, cnt, xs_gate,
+      xs_up, xs_down, g, u, acc_g, acc_u, acc_y, spmv, total;
 };
 inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   FfnWs w;
@@ -104,26 +107,29 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
     o = round_up(o + bytes, kAlign);
     return at;
   };
+  const bool one = B == 1;
   w.bar = take(sizeof(GridBarrier));
+  w.ctr = take(32);
   w.h = take((size_t)B * ffn * 4);
-  w.keys_d = take((size_t)B * ffn * 4);
-  w.idx_gate = take((size_t)B * d * 4);
-  w.idx_up = take((size_t)B * d * 4);
-  w.idx_down = take((size_t)B * ffn * 4);
-  w.cnt = take((size_t)3 * B * 4);
+  w.keep_g = take((size_t)B * d);
+  w.keep_u = take((size_t)B * d);
+  w.keep_d = take((size_t)B * ffn);
   w.stamps = take((size_t)kFfnStamps * 8);
   w.cta_t = take((size_t)kGridCap * 4 * 8);
-  w.xs_gate = take((size_t)B * d * 4);
-  w.xs_up = take((size_t)B * d * 4);
-  w.xs_down = take((size_t)B * ffn * 4);
-  w.g = take((size_t)B * ffn * 4);
-  w.u = take((size_t)B * ffn * 4);
-  const size_t gp = (size_t)kGridCap * ffn * 4, dp = (size_t)kGridCap * d * 4;
-  w.part_g = take(B == 1 ? gp : 0);
-  w.part_u = take(B == 1 ? gp : 0);
-  w.part_d = take(B == 1 ? dp : 0);
+  w.idx_gate = take(one ? 0 : (size_t)B * d * 4);
+  w.idx_up = take(one ? 0 : (size_t)B * d * 4);
+  w.idx_down = take(one ? 0 : (size_t)B * ffn * 4);
+  w.cnt = take(one ? 0 : (size_t)3 * B * 4);
+  w.xs_gate = take(one ? 0 : (size_t)B * d * 4);
+  w.xs_up = take(one ? 0 : (size_t)B * d * 4);
+  w.xs_down = take(one ? 0 : (size_t)B * ffn * 4);
+  w.g = take(one ? 0 : (size_t)B * ffn * 4);
+  w.u = take(one ? 0 : (size_t)B * ffn * 4);
+  w.acc_g = take(one ? (size_t)2 * ffn * 4 : 0);
+  w.acc_u = take(one ? (size_t)2 * ffn * 4 : 0);
+  w.acc_y = take(one ? (size_t)d * 4 : 0);
   const int64_t mmax = ffn > d ? ffn : d;
-  w.spmv = take(B == 1 ? 0 : spmv_ws_layout(mmax, B).total);
+  w.spmv = take(one ? 0 : spmv_ws_layout(mmax, B).total);
   w.total = o;
   return w;
 }

@@ -2,8 +2,9 @@
 //
 //  * wina_select_topk ("WINA" article, section 一): score_i = |x_i * c_i| in float32,
 //    keep the K largest (ties to the lower index), written as an ascending index list.
-//    One CTA per token: scores live in SMEM as uint32 bit patterns, a warp-ballot radix
-//    select finds the K-th largest, a two-walk warp-ballot compaction emits the list.
+//    One CTA per token: scores live in SMEM as uint32 bit patterns, a histogram select
+//    finds the K-th largest as a threshold, a two-walk warp-ballot compaction emits the
+//    kept indices in ascending order.
 //  * stat_topk_threshold ("Spark Transformer", section 2.2): mu, sigma^2 (divisor n) in
 //    one pass (Welford per thread, Chan's merge across threads, float64), then
 //    t = mu + sigma * z with z = Phi^-1(1 - s) from the host, keep {i : v_i > t}.
@@ -18,9 +19,10 @@ __global__ void __launch_bounds__(NT) k_select_topk(const void* __restrict__ x, 
                                                     int n, int K, int ld, int32_t* __restrict__ idx,
                                                     float* __restrict__ xs, float* __restrict__ scores) {
   extern __shared__ __align__(16) uint32_t sm[];
-  uint32_t* keys = sm;       // [n]
-  uint32_t* hist = sm + n;   // [512] select histograms
-  __shared__ uint32_t red[64];
+  uint32_t* keys = sm;                 // [n]
+  uint32_t* hist = sm + n;             // [kSelBins]
+  uint32_t* cand = hist + kSelBins;    // [2 * kSelCand]
+  __shared__ uint32_t red[2 * NT / 32 + 8];
   const int64_t b = blockIdx.x;
   const int64_t off = b * (int64_t)n;
   for (int i = threadIdx.x; i < n; i += NT) {
@@ -30,12 +32,19 @@ __global__ void __launch_bounds__(NT) k_select_topk(const void* __restrict__ x, 
     if (scores) scores[off + i] = s;
   }
   __syncthreads();
-  const Selection sel = select_topk_block<NT>(keys, n, K, hist);
+  const Threshold t = select_threshold<NT>(keys, n, K, hist, cand, red);
   const int64_t ob = b * (int64_t)ld;
-  compact_selection<NT>(keys, n, sel, 0u, (uint32_t)K, red, [&](int i, uint32_t pos) {
-    idx[ob + pos] = i;
-    if (xs) xs[ob + pos] = load_elem(x, xdt, off + i);
-  });
+  compact_pred<NT>(
+      n, [&](int i) { return kept_by(t, keys[i], i); },
+      [&](uint32_t, uint32_t* lo, uint32_t* hi) {
+        *lo = 0;
+        *hi = (uint32_t)K;
+      },
+      red,
+      [&](int i, uint32_t pos) {
+        idx[ob + pos] = i;
+        if (xs) xs[ob + pos] = load_elem(x, xdt, off + i);
+      });
 }
 
 template <int NT>
@@ -82,7 +91,7 @@ __global__ void __launch_bounds__(NT) k_stat_threshold(const void* __restrict__ 
 
 wina_status_t launch_select_topk(const void* x, int xdt, const float* c, int n, int k, int batch, int32_t* idx,
                                  float* xs, int ld, float* scores, cudaStream_t s) {
-  const size_t smem = (size_t)(n + 512) * 4;
+  const size_t smem = (size_t)(n + kSelBins + 2 * kSelCand) * 4;
   return cuda_status(launch_kernel(k_select_topk<kNT>, dim3(batch), dim3(kNT), smem, s, false, x, xdt, c, n, k, ld,
                                    idx, xs, scores));
 }

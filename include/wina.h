@@ -101,25 +101,22 @@ typedef struct {
 
 /* Byte offsets, inside the workspace of a sparse_ffn_swiglu call, of the intermediate
  * results it leaves behind (valid after the call completes; read-only diagnostics):
- *   h        float32 [batch][ffn]   h = silu(g) * u, the down projection's input
- *   idx_gate int32  [batch][d]      kept gate channels, ascending (first cnt_gate[b])
- *   idx_up   int32  [batch][d]      kept up channels, ascending
- *   idx_down int32  [batch][ffn]    kept down channels, ascending
- *   cnt      int32  [3][batch]      kept counts of gate, up and down per token
- *   stamps   int64  [16]            single-token kernel only: SM clock (clock64) of CTA 0
- *                                   at its phase boundaries: 0 start, 1 gate/up selected,
- *                                   2 gate/up rows streamed, 3 barrier, 4 h written,
- *                                   5 barrier, 6 down selected, 7 down rows streamed,
- *                                   8 barrier, 9 end
- *   cta_t    uint64 [CTAs][4]       single-token kernel only: global timer (ns) at which
- *                                   each CTA finished selecting gate/up, streaming
- *                                   gate/up rows, selecting down, streaming down rows   */
+ *   h         float32 [batch][ffn]  h = silu(g) * u, the down projection's input
+ *   keep_gate uint8   [batch][d]    1 where the gate projection's input channel was kept
+ *   keep_up   uint8   [batch][d]    1 where the up projection's input channel was kept
+ *   keep_down uint8   [batch][ffn]  1 where the down projection's input channel was kept
+ *   stamps    int64   [16]          single-token kernel only: SM clock (clock64) of CTA 0
+ *                                   at its phase boundaries: 0 start, 1 gate/up kept sets
+ *                                   known, 2 gate/up rows streamed, 3 barrier, 4 h written,
+ *                                   5 barrier, 6 down kept set known, 7 down rows
+ *                                   streamed, 8 barrier, 9 end
+ *   cta_t     uint64  [CTAs][4]     single-token kernel only: global timer (ns) at which
+ *                                   each CTA finished phases 1, 2, 6 and 7 above        */
 typedef struct {
   size_t h;
-  size_t idx_gate;
-  size_t idx_up;
-  size_t idx_down;
-  size_t cnt;
+  size_t keep_gate;
+  size_t keep_up;
+  size_t keep_down;
   size_t stamps;
   size_t cta_t;
 } wina_ffn_ws_view_t;
@@ -248,9 +245,11 @@ wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt, int64_t n,
  *   S_d = gate(h, c_down, k_down);  y = W_down[:, S_d] h[S_d]
  * With WINA_GATE_STAT every gate is the Spark threshold with keep fraction s on the
  * projection's signed input (k_* ignored); with WINA_GATE_DENSE every channel is kept.
- * One token runs as one persistent cooperative kernel (every SM selects redundantly
- * from x, streams its share of kept rows, and grid barriers separate the phases);
- * several tokens run as a sequence of the batched calls above.
+ * One token runs as one persistent cooperative kernel: each SM works on the gate or the
+ * up projection, selects that projection's kept channels itself, takes small units of
+ * channels from a global counter and streams their kept weight rows HBM -> SMEM with
+ * bulk copies through a ring of stages; grid barriers (bounded waits) separate the
+ * phases. Several tokens run as a sequence of the batched calls above.
  *   f:   host pointer to the weight descriptor (read during the call only).
  *   x:   device [batch][d] of xdt.   y: device float32 [batch][d] (written).
  *   k_gate, k_up in [0, d]; k_down in [0, ffn] (WINA_GATE_TOPK).  0 < s < 1 (STAT).

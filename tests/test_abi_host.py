@@ -53,7 +53,8 @@ def test_workspace_sizes():
     assert s1 >= 296 * 11008 * 4
     assert W.workspace_size(W.OP_SPARSE_MATVEC, 4096, 11008, 2048, 4096) < s1  # one CTA per token: no partials
     f1 = W.workspace_size(W.OP_FFN_SWIGLU, 4096, 11008, 0, 1)
-    assert f1 >= 296 * (2 * 11008 + 4096) * 4
+    assert f1 >= (2 * 2 * 11008 + 4096) * 4  # double-buffered g/u sums and the y sums
+    assert W.workspace_size(W.OP_FFN_SWIGLU, 4096, 11008, 0, 4) > f1  # several tokens: per-token buffers
     assert W.workspace_size(W.OP_SELECT_TOPK, 10, 10, 1, 1) == 0
     assert W.workspace_size(W.OP_FFN_SWIGLU, 0, 10, 0, 1) == 0
 
@@ -61,9 +62,8 @@ def test_workspace_sizes():
 def test_ffn_ws_view_offsets_are_disjoint():
     v = W._FfnView()
     assert W.lib.wina_ffn_ws_view(4096, 11008, 2, ctypes.byref(v)) == W.OK
-    spans = sorted([(v.h, 2 * 11008 * 4), (v.idx_gate, 2 * 4096 * 4), (v.idx_up, 2 * 4096 * 4),
-                    (v.idx_down, 2 * 11008 * 4), (v.cnt, 3 * 2 * 4), (v.stamps, 16 * 8),
-                    (v.cta_t, 296 * 4 * 8)])
+    spans = sorted([(v.h, 2 * 11008 * 4), (v.keep_gate, 2 * 4096), (v.keep_up, 2 * 4096),
+                    (v.keep_down, 2 * 11008), (v.stamps, 16 * 8), (v.cta_t, 296 * 4 * 8)])
     for (a, la), (b, _) in zip(spans, spans[1:]):
         assert a + la <= b
         assert a % 256 == 0

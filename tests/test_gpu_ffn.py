@@ -42,19 +42,17 @@ def _check_topk_ffn(f, Wgf, Wuf, Wdf, xb, x32, kg, ku, kd, batch=None):
     for b in range(B):
         ig = O.wina_select(x32[b], cg, kg)
         iu = O.wina_select(x32[b], cu, ku)
-        assert np.array_equal(v["idx_gate"][b][:kg], ig)
-        assert np.array_equal(v["idx_up"][b][:ku], iu)
+        assert np.array_equal(np.nonzero(v["keep_gate"][b])[0], ig)
+        assert np.array_equal(np.nonzero(v["keep_up"][b])[0], iu)
         x64 = x32[b].astype(np.float64)
         h_ref = O.silu(O.sparse_matvec(Wgf, ig, x64[ig])) * O.sparse_matvec(Wuf, iu, x64[iu])
         h_gpu = v["h"][b]
         assert rel_l2(h_gpu, h_ref) <= TOL_STAGE
         idn = O.wina_select(h_gpu, cd, kd)
-        assert np.array_equal(v["idx_down"][b][:kd], idn)
+        assert np.array_equal(np.nonzero(v["keep_down"][b])[0], idn)
         assert rel_l2(y[b], O.sparse_matvec(Wdf, idn, h_gpu[idn].astype(np.float64))) <= TOL_STAGE
         e2e = O.ffn_swiglu(Wgf, Wuf, Wdf, cg, cu, cd, x32[b], kg, ku, kd)
         assert rel_l2(y[b], e2e["y"]) <= TOL_E2E
-    if B == 1:
-        assert v["cnt"][:, 0].tolist() == [kg, ku, kd]
     return y
 
 
@@ -113,13 +111,21 @@ def test_llama7b_dense_mode(llama7b):
     assert rel_l2(y[0], O.dense_matvec(Wdf, h)) <= 1e-5
 
 
-def test_llama7b_deterministic(llama7b):
+def test_llama7b_repeatable(llama7b):
+    # The single-token kernel hands out work units dynamically, so the float32 summation
+    # order of the products (not the kept sets of gate and up) can change between calls:
+    # repeated calls must keep the same gate/up sets and agree to float32 rounding.
     cfg, f, *_ = llama7b
     ws = W.Workspace(W.OP_FFN_SWIGLU, 4096, 11008, 0, 1)
     xb = dev_bf16(cfg["x"][:1])
     a = host(W.sparse_ffn_swiglu(f, xb, W.GATE_TOPK, 2048, 2048, 5504, ws=ws))
-    for _ in range(3):
-        assert np.array_equal(a, host(W.sparse_ffn_swiglu(f, xb, W.GATE_TOPK, 2048, 2048, 5504, ws=ws)))
+    v0 = {k: host(t).copy() for k, t in W.ffn_ws_view(ws, 4096, 11008, 1).items()}
+    for _ in range(5):
+        b = host(W.sparse_ffn_swiglu(f, xb, W.GATE_TOPK, 2048, 2048, 5504, ws=ws))
+        v = W.ffn_ws_view(ws, 4096, 11008, 1)
+        assert np.array_equal(host(v["keep_gate"]), v0["keep_gate"])
+        assert np.array_equal(host(v["keep_up"]), v0["keep_up"])
+        assert rel_l2(b, a) <= 1e-5
 
 
 @pytest.mark.parametrize("d,ffn,dt", [(64, 128, "bf16"), (512, 1024, "f32"), (2304, 9216, "bf16"), (8, 16, "f32")])
@@ -165,19 +171,18 @@ def test_gemma_stat_gate(gemma, B):
     y = host(W.sparse_ffn_swiglu(f, dev_bf16(xb), W.GATE_STAT, s=s, ws=ws, status=st))
     assert int(host(st)[0]) == 0
     v = {k: host(t) for k, t in W.ffn_ws_view(ws, d, ffn, B).items()}
-    cnt = v["cnt"]
     for b in range(B):
         ref = O.spark_threshold(x32[b], s)
-        ig = v["idx_gate"][b][: cnt[0][b]]
+        ig = np.nonzero(v["keep_gate"][b])[0]
         diff = np.setxor1d(ig, ref["idx"])
         assert np.all(np.abs(x32[b][diff] - ref["t"]) <= 1e-5 * ref["sigma"])
-        assert np.array_equal(v["idx_up"][b][: cnt[1][b]], ig)
+        assert np.array_equal(np.nonzero(v["keep_up"][b])[0], ig)
         x64 = x32[b].astype(np.float64)
         h_ref = O.silu(O.sparse_matvec(Wgf, ig, x64[ig])) * O.sparse_matvec(Wuf, ig, x64[ig])
         h_gpu = v["h"][b]
         assert rel_l2(h_gpu, h_ref) <= TOL_STAGE
         rd = O.spark_threshold(h_gpu, s)
-        idn = v["idx_down"][b][: cnt[2][b]]
+        idn = np.nonzero(v["keep_down"][b])[0]
         diff = np.setxor1d(idn, rd["idx"])
         assert np.all(np.abs(h_gpu[diff] - rd["t"]) <= 1e-5 * rd["sigma"])
         assert rel_l2(y[b], O.sparse_matvec(Wdf, idn, h_gpu[idn].astype(np.float64))) <= TOL_STAGE

@@ -76,14 +76,14 @@ def test_llama3_ffn(llama3, B):
     for b in range(B):
         ig = O.wina_select(x32[b], cg, kg)
         iu = O.wina_select(x32[b], cu, ku)
-        assert np.array_equal(v["idx_gate"][b][:kg], ig)
-        assert np.array_equal(v["idx_up"][b][:ku], iu)
+        assert np.array_equal(np.nonzero(v["keep_gate"][b])[0], ig)
+        assert np.array_equal(np.nonzero(v["keep_up"][b])[0], iu)
         x64 = x32[b].astype(np.float64)
         h_rows = O.silu(O.sparse_matvec_rows(Wgr, ig, x64[ig])) * O.sparse_matvec_rows(Wur, iu, x64[iu])
         h_gpu = v["h"][b]
         assert rel_l2(h_gpu[grow], h_rows) <= 1e-5
         idn = O.wina_select(h_gpu, cd, kd)
-        assert np.array_equal(v["idx_down"][b][:kd], idn)
+        assert np.array_equal(np.nonzero(v["keep_down"][b])[0], idn)
         assert rel_l2(y[b][drow], O.sparse_matvec_rows(Wdr, idn, h_gpu[idn].astype(np.float64))) <= 1e-5
 
 
