@@ -613,6 +613,28 @@ __device__ void hist_crossing(const uint32_t* __restrict__ hist, uint32_t r, uin
   *cnt = s_cnt;
 }
 
+// The candidates cand[0..nc) = (key, index) pairs: set the flag bits of the r with the
+// highest (key desc, index asc). Warp w ranks candidates w, w + NT/32, ...: its lanes
+// compare that candidate with a 32-strided slice of the others each and sum the counts.
+// Ends with a block barrier.
+template <int NT>
+__device__ __forceinline__ void rank_and_keep(const uint32_t* __restrict__ cand, int nc, uint32_t r,
+                                              uint32_t* __restrict__ flags) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int c = warp; c < nc; c += NW) {
+    const uint32_t kc = cand[2 * c], ic = cand[2 * c + 1];
+    uint32_t above = 0u;
+    for (int o = lane; o < nc; o += 32) {
+      const uint32_t ko = cand[2 * o], io = cand[2 * o + 1];
+      above += (ko > kc || (ko == kc && io < ic)) ? 1u : 0u;
+    }
+    above = __reduce_add_sync(0xffffffffu, above);
+    if (lane == 0 && above < r) atomicOr(&flags[ic >> 5], 1u << (ic & 31));
+  }
+  __syncthreads();
+}
+
 // Kept-channel bitmask of the exact top-K of keys[0..n) in SMEM (ties to the lower
 // index), given the keys' min and max. One histogram pass over a linear map of the key
 // bits onto kSelBins bins (monotone, so bins are ordered like the keys), a two-level
@@ -677,19 +699,94 @@ __device__ void select_topk_flags(const uint32_t* __restrict__ keys, int n, int 
     }
   }
   __syncthreads();
-  const int nc = (int)s_ncand;
-  for (int c = threadIdx.x; c < nc; c += NT) {
-    const uint32_t kc = cand[2 * c];
-    const int ic = (int)cand[2 * c + 1];
-    uint32_t rank = 0u;
-    for (int o = 0; o < nc; ++o) {
-      const uint32_t ko = cand[2 * o];
-      const int io = (int)cand[2 * o + 1];
-      rank += (ko > kc || (ko == kc && io < ic)) ? 1u : 0u;
+  rank_and_keep<NT>(cand, (int)s_ncand, r, flags);
+}
+
+// Kept-channel bitmask of the exact top-K of keys[0..n) in SMEM (ties to the lower
+// index), given hist = the counts of the keys' top 12 bits (key >> 19; bit 31 of a
+// non-negative float is 0), which the caller fills while it produces the keys. A
+// two-level scan finds the bin holding the K-th key; one pass sets the flags of every
+// channel outside that bin and gathers the bin's keys, which are ranked exactly. If the
+// bin holds more than kSelCand keys, the general search (select_threshold) decides.
+// flags[w] bit l = channel 32w + l is kept. SMEM: keys 16-byte aligned and readable
+// up to the next multiple of 128 entries (the excess is ignored), hist [kSelBins]
+// (filled), cand [2 * kSelCand], red [>= 2 * NT/32 + 8]. Every thread of the block
+// must call it.
+template <int NT>
+__device__ void select_topk_flags_radix(const uint32_t* __restrict__ keys, int n, int K, uint32_t* __restrict__ hist,
+                                        uint32_t* __restrict__ cand, uint32_t* __restrict__ red,
+                                        uint32_t* __restrict__ flags, long long* st = nullptr) {
+  static_assert(kSelBins == 4096, "12-bit digit");
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = (n + 31) / 32;
+  __shared__ uint32_t s_ncand;
+  if (K <= 0 || K >= n) {
+    const int keep = K <= 0 ? 0 : n;
+    for (int w = threadIdx.x; w < nw; w += NT) {
+      const int rem = keep - w * 32;
+      flags[w] = rem >= 32 ? 0xffffffffu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
     }
-    if (rank < r) atomicOr(&flags[ic >> 5], 1u << (ic & 31));
+    __syncthreads();
+    return;
+  }
+  if (threadIdx.x == 0) s_ncand = 0u;
+  __syncthreads();  // the caller's histogram updates are complete
+  int B;
+  uint32_t above, cnt;
+  hist_crossing<NT>(hist, (uint32_t)K, red, &B, &above, &cnt);
+  if (st && threadIdx.x == 0) st[0] = clock64();
+  if (cnt > (uint32_t)kSelCand) {
+    const Threshold t = select_threshold<NT>(keys, n, K, hist, cand, red);
+    for (int w = warp; w < nw; w += NW) {
+      const int j = w * 32 + lane;
+      const uint32_t bits = __ballot_sync(0xffffffffu, j < n && kept_by(t, keys[j], j));
+      if (lane == 0) flags[w] = bits;
+    }
+    __syncthreads();
+    return;
+  }
+  const uint32_t r = (uint32_t)K - above;  // kept among the bin's keys
+  // flags outside the boundary bin, and the bin's keys gathered: each lane takes four
+  // consecutive channels (one 16-byte load), so a warp covers four flag words per step;
+  // eight lanes' nibbles are merged into a word by shuffles
+  const int n128 = (n + 127) / 128;
+  for (int q = warp; q < n128; q += NW) {
+    const int j0 = q * 128 + lane * 4;
+    const uint4 k4 = reinterpret_cast<const uint4*>(keys)[q * 32 + lane];
+    const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+    uint32_t nib = 0u, inb[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool in = j0 + e < n;
+      const int bj = (int)(kk[e] >> 19);
+      nib |= (in && bj > B) ? (1u << e) : 0u;
+      inb[e] = __ballot_sync(0xffffffffu, in && bj == B);
+    }
+    uint32_t v = nib << (4 * (lane & 7));
+    v |= __shfl_xor_sync(0xffffffffu, v, 1);
+    v |= __shfl_xor_sync(0xffffffffu, v, 2);
+    v |= __shfl_xor_sync(0xffffffffu, v, 4);
+    if ((lane & 7) == 0 && q * 4 + (lane >> 3) < nw) flags[q * 4 + (lane >> 3)] = v;
+    const uint32_t tot = __popc(inb[0]) + __popc(inb[1]) + __popc(inb[2]) + __popc(inb[3]);
+    if (tot) {  // uniform across the warp
+      const uint32_t lt = (1u << lane) - 1u;
+      uint32_t base = 0u;
+      if (lane == 0) base = atomicAdd(&s_ncand, tot);
+      base = __shfl_sync(0xffffffffu, base, 0) + __popc(inb[0] & lt) + __popc(inb[1] & lt) + __popc(inb[2] & lt) +
+             __popc(inb[3] & lt);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((inb[e] >> lane) & 1u) {
+          cand[2 * base] = kk[e];
+          cand[2 * base + 1] = (uint32_t)(j0 + e);
+          ++base;
+        }
+    }
   }
   __syncthreads();
+  if (st && threadIdx.x == 0) st[1] = clock64();
+  rank_and_keep<NT>(cand, (int)s_ncand, r, flags);
 }
 
 // ------------------------------------------------------------------------------------

@@ -8,17 +8,19 @@
 //      against its projection's c in SMEM, finds the K-th largest score by radix select
 //      (or the Spark threshold, or keeps everything) and turns the result into a
 //      kept-channel bitmask.
-//   B  The producer warp takes units of a few channels from a global counter (dynamic
-//      load balance across the CTAs of the projection), and for each kept channel
-//      copies the whole input-major weight row HBM -> SMEM with a bulk copy into a ring
-//      of stages (full/empty mbarriers). Consumer warps accumulate x_j * row_j in
-//      float32 registers and finally store one partial row per CTA.
-//      At the end each CTA adds its row sums into g or u (vector float atomics at L2).
+//   B  The producer warp streams the kept input-major weight rows HBM -> SMEM with bulk
+//      copies into a ring of stages (full/empty mbarriers): first the CTA's own block of
+//      channels, then units of a few channels from a global counter (dynamic load
+//      balance across the CTAs of the projection). Consumer warps accumulate x_j * row_j
+//      in float32 registers; at the end each CTA adds its row sums into g or u (vector
+//      float atomics at L2).
 //   -- grid barrier --
 //   C  Every CTA reads the complete g and u, computes h = silu(g) * u and the down
 //      gate's scores |h_j * c_down_j| for all ffn channels, and selects the kept down
 //      channels itself (bitmask).
-//   E  As B, over the down projection's rows (d wide), all CTAs together; row sums are
+//   E  Every CTA takes an equal share of the kept down rows (by rank in index order)
+//      and streams them with 16-byte loads, 16 rows in flight per thread (rows of d
+//      elements are too short for bulk copies to reach HBM bandwidth); row sums are
 //      added into y's accumulator.
 //   F  The last CTA to finish (a counter) copies y out and clears the accumulators.
 // Every wait (grid barrier, ring stage) is bounded in time; on a timeout the kernel
@@ -56,10 +58,13 @@ struct FfnParams {
   double z;
   float* y;
   int Gg;             // CTAs on the gate projection in phase B
-  int uw_b, uw_e;     // channels per work unit in phases B and E
-  int S_b, S_e;       // ring stages in phases B and E
+  int cs_g, cs_u, cs_e;  // channels in each CTA's own block: gate, up (phase B), down (E)
+  int wmin_b, wmin_e;    // shortest dynamic unit (channels) in phases B and E
+  int rows_e;            // phase E: rows per ring stage (longest contiguous copy)
+  int smem;              // dynamic SMEM bytes of the launch
+  int S_b;            // ring stages in phase B
   GridBarrier* bar;
-  unsigned* ctr;  // [3] unit counters: gate, up, down
+  unsigned* ctr;  // [3] channel counters of the dynamic units: gate, up, down
   float* h;
   uint8_t* keep_g;
   uint8_t* keep_u;
@@ -76,14 +81,18 @@ struct FfnParams {
 };
 
 struct SmemLayout {
-  uint32_t keys, vals, flags, meta_val, meta_row, bars, ring, hist, cand;
+  uint32_t vals, flags, meta_row, meta_cnt, bars, keys, ring, hist, cand, stage;
 };
 
-// keys | vals | flags | stage metadata | mbarriers | ring. The selection's histogram and
-// candidate list overlay the start of the ring, which is idle while a selection runs.
+// vals | flags | stage metadata | mbarriers | keys | ring. The selection's histogram and
+// candidate list, and the input staging buffer, overlay the start of the ring, which is
+// idle while a selection runs; in phase E the ring extends down over keys (past the
+// CTA's row list kept at its start).
 __host__ __device__ inline SmemLayout ffn_smem_layout(int d, int ffn) {
   SmemLayout L;
-  const uint32_t nb = (uint32_t)(d > ffn ? d : ffn);
+  // room for max(d, ffn) channels, rounded up to 128 (the selection reads whole
+  // 128-channel blocks)
+  const uint32_t nb = ((uint32_t)(d > ffn ? d : ffn) + 127u) / 128u * 128u;
   uint32_t o = 0;
   auto take = [&](uint32_t bytes, uint32_t align) {
     o = (o + align - 1) / align * align;
@@ -91,22 +100,33 @@ __host__ __device__ inline SmemLayout ffn_smem_layout(int d, int ffn) {
     o += bytes;
     return at;
   };
-  L.keys = take(nb * 4, 16);
   L.vals = take(nb * 4, 16);
   L.flags = take((nb + 31) / 32 * 4, 16);
-  L.meta_val = take(kMaxStages * 4, 16);
   L.meta_row = take(kMaxStages * 4, 16);
-  L.bars = take(2 * kMaxStages * 8, 16);
+  L.meta_cnt = take(kMaxStages * 4, 16);
+  L.bars = take((2 * kMaxStages + 1) * 8, 16);
+  L.keys = take(nb * 4, 128);
   L.ring = take(0, 128);
   L.hist = L.ring;
   L.cand = L.ring + kSelBins * 4;
+  L.stage = L.cand + 2 * kSelCand * 4;  // 16-byte aligned input staging
   return L;
 }
 
-// Smallest ring the layout needs (the selection scratch lives in it).
-constexpr uint32_t kMinRing = (kSelBins + 2 * kSelCand) * 4;
+// Smallest ring the layout needs: the selection scratch and an input staging buffer of
+// max(d, ffn) float32 live in it while a selection runs.
+__host__ __device__ inline uint32_t ffn_min_ring(int d, int ffn) {
+  return (uint32_t)((kSelBins + 2 * kSelCand) * 4) + (uint32_t)(d > ffn ? d : ffn) * 4;
+}
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+// One L2 prefetch per 2 MB of [p, p + bytes), spread over the CTA's threads.
+__device__ __forceinline__ void touch_pages(const void* p, size_t bytes) {
+  const char* c = reinterpret_cast<const char*>(p);
+  for (size_t o = (size_t)threadIdx.x << 21; o < bytes; o += (size_t)kFT << 21)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(c + o));
+}
 
 // CTA 0 records its SM clock at phase boundaries; every CTA records the global timer at
 // the end of its four main phases (diagnostic views of the workspace).
@@ -175,13 +195,17 @@ __device__ double spark_threshold(const float* v, int n, double z, double* dred)
 // ------------------------------------------------------------------------------------
 // the row ring: producer and consumers
 // ------------------------------------------------------------------------------------
+// Kept channels that follow one another have adjacent rows in the input-major layout.
+// A stage holds a piece of up to `rmax` such rows, fetched by one bulk copy: bulk copies
+// of short rows at scattered addresses stream well below HBM bandwidth, contiguous
+// copies of 16 KB and more reach it (so rmax > 1 for the short down rows).
 
 struct Ring {
   char* base;      // SMEM
   uint64_t* full;  // [kMaxStages]
   uint64_t* empty;  // [kMaxStages]
-  float* meta_val;  // x_j (or h_j) of the row in each stage
-  int* meta_row;    // row index of each stage, -1 = end of phase
+  int* meta_row;    // first row of the piece in each stage, -1 = end of phase
+  int* meta_cnt;    // rows in the piece
 };
 
 // Producer state kept across phases (per-stage mbarrier parities).
@@ -191,81 +215,131 @@ struct ProdState {
   uint32_t full_par;   // parity of the next phase on full[s] (last issued = bit ^ 1)
 };
 
-// Streams the kept rows of channels [0, n) unit by unit (units of `uw` <= 32 channels
-// taken from the global counter `ctr`) into the ring, then an end-of-phase marker. Runs
-// on the producer warp. The kept rows of a unit are issued by as many lanes at once (a
-// single thread issuing bulk copies one after another is far too slow to fill HBM), in
-// rounds of at most S rows so that the stages of a round are distinct. Lane 0 keeps
-// kGrab unit requests in flight, each in its own register, so that a request's counter
-// round trip is waited on only when that unit is next (a shuffle of a register with a
-// load still pending would stall on it). Returns false on a timeout.
-constexpr int kGrab = 2;
-__device__ bool produce(const Ring& R, int S, uint32_t row_bytes, const char* __restrict__ Wt, int n, int uw,
-                        unsigned* ctr, const uint32_t* flags, const float* vals, ProdState& ps, uint64_t pol,
-                        unsigned long long* trace = nullptr) {
+// Work of one phase for the producer warp: kept rows of channels [0, n), the CTA's own
+// block [s0, s1) first, then units over [base, n) taken from the global channel counter
+// `ctr` (dynamic load balance). Unit widths are guided: the part of [base, n) not yet
+// handed out divided by 2 * `parts` (the CTAs sharing the counter), clamped to
+// [wmin, 32], so that units are long while much is left and short at the end.
+struct PhaseWork {
+  int n, s0, s1, base, parts, wmin;
+  unsigned* ctr;
+};
+
+// Streams the phase's kept rows into the ring in pieces (see above), then an end-of-
+// phase marker. Runs on the producer warp. The pieces of a 32-channel window are issued
+// by as many lanes at once (a single thread issuing bulk copies one after another is
+// far too slow to fill HBM), in rounds of at most S so that the stages of a round are
+// distinct. The next unit is requested when a unit starts, so the counter's round trip
+// overlaps the unit's copies, and none is requested while the CTA's own block is
+// streamed. Returns false on a timeout.
+__device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage_bytes, int rmax,
+                        const char* __restrict__ Wt, const PhaseWork& wk, const uint32_t* flags, ProdState& ps,
+                        uint64_t pol, unsigned long long* trace = nullptr) {
   const int lane = threadIdx.x & 31;
-  const uint32_t lt = (1u << lane) - 1u;
-  const unsigned nunits = (unsigned)((n + uw - 1) / uw);
+  const uint32_t lt = (1u << lane) - 1u, le = lt | (1u << lane);
   int stage = 0;
-  unsigned pend[kGrab];
-#pragma unroll
-  for (int q = 0; q < kGrab; ++q) pend[q] = lane == 0 ? atomicAdd(ctr, 1u) : 0u;
-  uint32_t live = (1u << kGrab) - 1u;
-  bool ok = true;
-  while (live) {
-#pragma unroll
-    for (int q = 0; q < kGrab; ++q) {
-      if (!((live >> q) & 1u)) continue;  // uniform across the warp
-      unsigned unit = lane == 0 ? pend[q] : 0u;
-      unit = __shfl_sync(0xffffffffu, unit, 0);
-      if (unit >= nunits) {
-        live &= ~(1u << q);
-        continue;
-      }
-      if (lane == 0) pend[q] = atomicAdd(ctr, 1u);  // refill this request
-      const int j0 = (int)unit * uw;
-      const int j = j0 + lane;
-      const bool k = lane < uw && j < n && ((flags[j >> 5] >> (j & 31)) & 1u);
-      const uint32_t m = __ballot_sync(0xffffffffu, k);
-      const int cnt = __popc(m);
-      const int pos = __popc(m & lt);
-      for (int r0 = 0; r0 < cnt; r0 += S) {
-        const int nr = min(S, cnt - r0);
-        if (k && pos >= r0 && pos < r0 + nr) {
-          const int s = (stage + pos - r0) % S;
-          bool mine_ok = true;
-          if ((ps.used >> s) & 1u) mine_ok = mbar_wait(&R.empty[s], (ps.empty_par >> s) & 1u);
-          if (mine_ok) {
-            R.meta_val[s] = vals[j];
-            R.meta_row[s] = j;
-            mbar_arrive_expect_tx(&R.full[s], row_bytes);
-            bulk_copy_g2s(R.base + (size_t)s * row_bytes, Wt + (size_t)j * row_bytes, row_bytes, &R.full[s], pol);
-            if (trace && stage + pos - r0 < 64) trace[stage + pos - r0] = globaltimer_ns();
-          } else {
+  // kept rows of channels [j0, j1), j1 - j0 <= 32
+  auto issue = [&](int j0, int j1) {
+    const int j = j0 + lane;
+    const bool k = j < j1 && ((flags[j >> 5] >> (j & 31)) & 1u);
+    const uint32_t km = __ballot_sync(0xffffffffu, k);
+    const uint32_t runs = km & ~(km << 1);                 // first lanes of runs of kept channels
+    const int rs = 31 - __clz(runs & le);                  // start of this lane's run (if kept)
+    const bool head = k && ((lane - rs) % rmax == 0);      // first lane of a piece
+    const uint32_t heads = __ballot_sync(0xffffffffu, head);
+    const uint32_t after = (heads | ~km) & ~le;
+    const int len = (after ? __ffs(after) - 1 : 32) - lane;  // rows in the piece headed here
+    const int np = __popc(heads), pos = __popc(heads & lt);
+    bool ok = true;
+    for (int r0 = 0; r0 < np; r0 += S) {
+      const int nr = min(S, np - r0);
+      // each lane issues its piece as soon as its stage is free (the oldest first), so
+      // the ring is refilled stage by stage rather than a round at a time
+      bool mine = head && pos >= r0 && pos < r0 + nr;
+      const int s = (stage + pos - r0) % S;
+      const bool was_used = (ps.used >> s) & 1u;
+      const uint32_t par = (ps.empty_par >> s) & 1u;
+      unsigned long long t0 = 0;
+      while (__any_sync(0xffffffffu, mine)) {
+        if (!mine) continue;
+        if (!was_used || mbar_try_wait(&R.empty[s], par)) {
+          const uint32_t bytes = (uint32_t)len * row_bytes;
+          R.meta_row[s] = j;
+          R.meta_cnt[s] = len;
+          mbar_arrive_expect_tx(&R.full[s], bytes);
+          bulk_copy_g2s(R.base + (size_t)s * stage_bytes, Wt + (size_t)j * row_bytes, bytes, &R.full[s], pol);
+          if (trace && stage + pos - r0 < 64) trace[stage + pos - r0] = globaltimer_ns();
+          mine = false;
+        } else {
+          const unsigned long long now = globaltimer_ns();
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > kPipeTimeoutNs) {
             ok = false;
+            mine = false;
           }
         }
-        // the same state update in every lane: nr consecutive stages were filled
-        for (int i = 0; i < nr; ++i) {
-          const int s = (stage + i) % S;
-          if ((ps.used >> s) & 1u) ps.empty_par ^= 1u << s;
-          ps.used |= 1u << s;
-          ps.full_par ^= 1u << s;
-        }
-        stage += nr;
-        if (__any_sync(0xffffffffu, !ok)) return false;
+      }
+      // the same state update in every lane: nr consecutive stages were filled
+      for (int i = 0; i < nr; ++i) {
+        const int s = (stage + i) % S;
+        if ((ps.used >> s) & 1u) ps.empty_par ^= 1u << s;
+        ps.used |= 1u << s;
+        ps.full_par ^= 1u << s;
+      }
+      stage += nr;
+      if (__any_sync(0xffffffffu, !ok)) return false;
+    }
+    return true;
+  };
+  bool ok = true;
+  const unsigned ndyn = wk.base < wk.n ? (unsigned)(wk.n - wk.base) : 0u;
+  auto width = [&](unsigned taken) {
+    const unsigned left = taken < ndyn ? ndyn - taken : 0u;
+    return (unsigned)min(32, max(wk.wmin, (int)(left / (2u * (unsigned)wk.parts))));
+  };
+  // the first unit is requested halfway through the CTA's own block, so that its round
+  // trip is hidden and it is not held long
+  unsigned pw = 0u, pstart = 0u;
+  const int half = wk.s0 + (wk.s1 - wk.s0) / 2;
+  bool asked = false;
+  for (int c = wk.s0; c < wk.s1 && ok; c += 32) {
+    if (!asked && c + 32 > half) {
+      if (lane == 0 && ndyn) {
+        pw = width(0u);
+        pstart = atomicAdd(wk.ctr, pw);
+      }
+      asked = true;
+    }
+    ok = issue(c, min(wk.s1, c + 32));
+  }
+  if (ok && ndyn) {
+    if (!asked && lane == 0) {
+      pw = width(0u);
+      pstart = atomicAdd(wk.ctr, pw);
+    }
+    while (true) {
+      const unsigned start = __shfl_sync(0xffffffffu, pstart, 0), w = __shfl_sync(0xffffffffu, pw, 0);
+      if (start >= ndyn) break;
+      if (lane == 0) {  // the next unit, while this one streams
+        pw = width(start + w);
+        pstart = atomicAdd(wk.ctr, pw);
+      }
+      const int j0 = wk.base + (int)start;
+      if (!issue(j0, min(wk.n, j0 + (int)w))) {
+        ok = false;
+        break;
       }
     }
   }
+  if (!__all_sync(0xffffffffu, ok)) return false;
   // end-of-phase marker: completes a stage with no bytes
   if (lane == 0) {
     const int s = stage % S;
-    if ((ps.used >> s) & 1u) {
-      if (!mbar_wait(&R.empty[s], (ps.empty_par >> s) & 1u)) ok = false;
-    }
+    if ((ps.used >> s) & 1u) ok = mbar_wait(&R.empty[s], (ps.empty_par >> s) & 1u);
     if (ok) {
-      R.meta_val[s] = 0.f;
       R.meta_row[s] = -1;
+      R.meta_cnt[s] = 0;
       mbar_arrive(&R.full[s]);
     }
   }
@@ -286,65 +360,63 @@ __device__ void drain(const Ring& R, const ProdState& ps) {
     if ((ps.used >> s) & 1u) mbar_wait(&R.full[s], ((ps.full_par >> s) & 1u) ^ 1u);
 }
 
-// Consumer warps: take stages in order until the end marker, accumulating
-// meta_val * row into acc (thread t owns 16-byte vectors t, t + kCT, ...).
-template <bool BF16, int VPT>
-__device__ bool consume_t(const Ring& R, int S, uint32_t row_bytes, int V, uint32_t& full_par,
-                          float (&acc)[VPT][VecOps<BF16>::EPV], unsigned long long* trace, int& rows) {
-  const int t = threadIdx.x, lane = t & 31;
-  const uint32_t ring = smem_addr(R.base);
-  int stage = 0;
-  while (true) {
-    const int s = stage % S;
-    if (!mbar_wait(&R.full[s], (full_par >> s) & 1u)) return false;
-    if (trace && t == 0 && stage < 64) trace[64 + stage] = globaltimer_ns();
-    full_par ^= 1u << s;
-    const int row = R.meta_row[s];
-    if (row >= 0) {
-      ++rows;
-      const float xv = R.meta_val[s];
-      const uint32_t src = ring + (uint32_t)s * row_bytes;
-      uint4 w[VPT];
-#pragma unroll
-      for (int j = 0; j < VPT; ++j) {
-        const int v = t + j * kCT;
-        if (v < V) w[j] = ld_shared_u4(src + (uint32_t)v * 16u);
-      }
-#pragma unroll
-      for (int j = 0; j < VPT; ++j) {
-        const int v = t + j * kCT;
-        if (v < V) VecOps<BF16>::fma(acc[j], w[j], xv);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&R.empty[s]);
-    if (row < 0) return true;
-    ++stage;
-  }
-}
-
 __device__ __forceinline__ void red_add_f4(float* p, float a, float b, float c, float d) {
   asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
 
-// Consume one phase, then add the CTA's float32 row sums into out[0..m) (vector
-// atomics at L2; the order of the CTAs' additions is not fixed).
+// Consumer warps: take stages in order until the end marker; for each row r of a stage,
+// acc += vals[meta_row + r] * row (thread t owns 16-byte vectors t, t + kCT, ...); then
+// add the row sums into out[0..m) (vector float atomics at L2; the order of the CTAs'
+// additions is not fixed). Returns false on a timeout.
 template <bool BF16, int VPT>
-__device__ bool consume_store_t(const Ring& R, int S, uint32_t row_bytes, int V, uint32_t& full_par,
-                                float* __restrict__ out, unsigned long long* trace) {
+__device__ bool consume_t(const Ring& R, int S, uint32_t row_bytes, uint32_t stage_bytes, int V, uint32_t& full_par,
+                          const float* vals, float* __restrict__ out, unsigned long long* trace) {
   constexpr int EPV = VecOps<BF16>::EPV;
+  const int t = threadIdx.x, lane = t & 31;
   float acc[VPT][EPV];
 #pragma unroll
   for (int j = 0; j < VPT; ++j)
 #pragma unroll
     for (int e = 0; e < EPV; ++e) acc[j][e] = 0.f;
-  int rows = 0;
-  const bool ok = consume_t<BF16, VPT>(R, S, row_bytes, V, full_par, acc, trace, rows);
+  const uint32_t ring = smem_addr(R.base);
+  int stage = 0, rows = 0;
+  bool ok = true;
+  while (true) {
+    const int s = stage % S;
+    if (!mbar_wait(&R.full[s], (full_par >> s) & 1u)) {
+      ok = false;
+      break;
+    }
+    if (trace && t == 0 && stage < 64) trace[64 + stage] = globaltimer_ns();
+    full_par ^= 1u << s;
+    const int row = R.meta_row[s];
+    if (row >= 0) {
+      const int nr = R.meta_cnt[s];
+      rows += nr;
+      const uint32_t src = ring + (uint32_t)s * stage_bytes;
+      for (int r = 0; r < nr; ++r) {
+        const float xv = vals[row + r];
+        uint4 w[VPT];
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+          const int v = t + j * kCT;
+          if (v < V) w[j] = ld_shared_u4(src + (uint32_t)r * row_bytes + (uint32_t)v * 16u);
+        }
+#pragma unroll
+        for (int j = 0; j < VPT; ++j)
+          if (t + j * kCT < V) VecOps<BF16>::fma(acc[j], w[j], xv);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&R.empty[s]);
+    if (row < 0) break;
+    ++stage;
+  }
   if (rows == 0) return ok;  // nothing to add
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
-    const int v = threadIdx.x + j * kCT;
+    const int v = t + j * kCT;
     if (v < V) {
       float* o = out + (int64_t)v * EPV;
 #pragma unroll
@@ -356,22 +428,19 @@ __device__ bool consume_store_t(const Ring& R, int S, uint32_t row_bytes, int V,
   return ok;
 }
 
-// Consume one phase and store the CTA's partial row out[0..m).
 template <bool BF16>
-__device__ bool consume_store(const Ring& R, int S, uint32_t row_bytes, int m, uint32_t& full_par, float* out,
-                              unsigned long long* trace = nullptr) {
+__device__ bool consume(const Ring& R, int S, uint32_t row_bytes, uint32_t stage_bytes, int m, uint32_t& full_par,
+                        const float* vals, float* out, unsigned long long* trace = nullptr) {
   constexpr int EPV = VecOps<BF16>::EPV;
   const int V = m / EPV;
-  const int vpt = (V + kCT - 1) / kCT;
-  switch (vpt) {
-    case 1: return consume_store_t<BF16, 1>(R, S, row_bytes, V, full_par, out, trace);
-    case 2: return consume_store_t<BF16, 2>(R, S, row_bytes, V, full_par, out, trace);
-    case 3: return consume_store_t<BF16, 3>(R, S, row_bytes, V, full_par, out, trace);
-    case 4: return consume_store_t<BF16, 4>(R, S, row_bytes, V, full_par, out, trace);
-    case 5: return consume_store_t<BF16, 5>(R, S, row_bytes, V, full_par, out, trace);
-    case 6: return consume_store_t<BF16, 6>(R, S, row_bytes, V, full_par, out, trace);
-    case 7: return consume_store_t<BF16, 7>(R, S, row_bytes, V, full_par, out, trace);
-    default: return consume_store_t<BF16, 8>(R, S, row_bytes, V, full_par, out, trace);
+  switch ((V + kCT - 1) / kCT) {
+    case 1: return consume_t<BF16, 1>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
+    case 2: return consume_t<BF16, 2>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
+    case 3: return consume_t<BF16, 3>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
+    case 4: return consume_t<BF16, 4>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
+    case 5: return consume_t<BF16, 5>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
+    case 6: return consume_t<BF16, 6>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
+    default: return consume_t<BF16, 8>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
   }
 }
 
@@ -391,11 +460,13 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   uint32_t* hist = reinterpret_cast<uint32_t*>(smraw + SL.hist);
   uint32_t* cand = reinterpret_cast<uint32_t*>(smraw + SL.cand);
   Ring R;
-  R.meta_val = reinterpret_cast<float*>(smraw + SL.meta_val);
   R.meta_row = reinterpret_cast<int*>(smraw + SL.meta_row);
+  R.meta_cnt = reinterpret_cast<int*>(smraw + SL.meta_cnt);
   R.full = reinterpret_cast<uint64_t*>(smraw + SL.bars);
   R.empty = R.full + kMaxStages;
   R.base = reinterpret_cast<char*>(smraw + SL.ring);
+  uint64_t* aux = R.full + 2 * kMaxStages;  // input staging copies
+  unsigned char* stage_in = smraw + SL.stage;
   __shared__ uint32_t red[2 * kFT / 32 + 8];
   __shared__ double dred[3 * kFT / 32];
   __shared__ int s_abort, s_last;
@@ -411,9 +482,11 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       mbar_init(&R.full[s], 1u);
       mbar_init(&R.empty[s], (uint32_t)kCW);
     }
+    mbar_init(aux, 1u);
     mbar_init_fence();
     s_abort = 0;
   }
+  __syncthreads();
   ProdState ps{0u, 0u, 0u};
   uint32_t full_par = 0u;
 
@@ -437,36 +510,45 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   const int rank = gate ? b : b - a.Gg;
   const float* cproj = gate ? a.c_gate : a.c_up;
   {
-    // all of this thread's loads are issued before any SMEM store (a store through a
-    // generic pointer could alias the inputs, which would serialise the round trips)
-    constexpr int U = 8;
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int i0 = threadIdx.x; i0 < d; i0 += U * kFT) {
-      float xv[U], cv[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = i0 + u * kFT;
-        xv[u] = i < d ? load_elem(a.x, a.xdt, i) : 0.f;
-        cv[u] = (i < d && a.mode == WINA_GATE_TOPK) ? __ldg(cproj + i) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = i0 + u * kFT;
-        if (i < d) {
-          vals[i] = xv[u];
-          if (a.mode == WINA_GATE_TOPK) {
-            const uint32_t k = __float_as_uint(fabsf(xv[u] * cv[u]));
-            keys[i] = k;
-            kmin = min(kmin, k);
-            kmax = max(kmax, k);
-          }
-        }
+    // x and this projection's c arrive by bulk copies (x into the staging buffer, c into
+    // the keys buffer, where each score then replaces its c in place); meanwhile the
+    // histogram is cleared. An x that is not 16-byte aligned is loaded by the threads.
+    const bool topk = a.mode == WINA_GATE_TOPK;
+    const uint32_t xbytes = (uint32_t)d * (a.xdt == WINA_BF16 ? 2u : 4u);
+    const bool xbulk = ((uintptr_t)a.x & 15u) == 0;
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(aux, (xbulk ? xbytes : 0u) + (topk ? (uint32_t)d * 4u : 0u));
+      if (xbulk) bulk_copy_g2s(stage_in, a.x, xbytes, aux, pol);
+      if (topk) bulk_copy_g2s(keys, cproj, (uint32_t)d * 4u, aux, pol);
+    }
+    // touch every 2 MB page of this projection's weights now, so that the address
+    // translations are warm when the rows stream (the first rows land later otherwise)
+    touch_pages(gate ? a.wt_gate : a.wt_up, (size_t)d * ffn * ESZ);
+    for (int i = threadIdx.x; i < kSelBins; i += kFT) hist[i] = 0u;
+    if (!xbulk)
+      for (int i = threadIdx.x; i < d; i += kFT) reinterpret_cast<float*>(stage_in)[i] = load_elem(a.x, a.xdt, i);
+    if (!mbar_wait(aux, 0u)) s_abort = 1;
+    __syncthreads();
+    if (s_abort) {
+      record_status(a.status, WINA_ERR_TIMEOUT);
+      return;
+    }
+    stamp(a.stamps, 10);
+    const bool xf32 = !xbulk || a.xdt == WINA_F32;
+    for (int i = threadIdx.x; i < d; i += kFT) {
+      const float xv = xf32 ? reinterpret_cast<const float*>(stage_in)[i]
+                            : bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(stage_in)[i]);
+      vals[i] = xv;
+      if (topk) {
+        const uint32_t k = __float_as_uint(fabsf(xv * __uint_as_float(keys[i])));
+        keys[i] = k;
+        atomicAdd(&hist[k >> 19], 1u);
       }
     }
-    if (a.mode == WINA_GATE_TOPK) {
-      uint32_t mn, mx;
-      block_minmax_u32<kFT>(kmin, kmax, red, mn, mx);  // contains the barrier after the loads
-      select_topk_flags<kFT>(keys, d, gate ? a.k_gate : a.k_up, mn, mx, hist, cand, red, flags);
+    stamp(a.stamps, 11);
+    if (topk) {
+      select_topk_flags_radix<kFT>(keys, d, gate ? a.k_gate : a.k_up, hist, cand, red, flags,
+                                   b == 0 ? a.stamps + 12 : nullptr);
     } else {
       __syncthreads();
       if (a.mode == WINA_GATE_STAT)
@@ -484,12 +566,18 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   {
     const uint32_t row_bytes = (uint32_t)ffn * ESZ;
     if (producer) {
-      const bool ok = produce(R, a.S_b, row_bytes, reinterpret_cast<const char*>(gate ? a.wt_gate : a.wt_up), d,
-                              a.uw_b, a.ctr + (gate ? 0 : 1), flags, vals, ps, pol, b == 0 ? a.trace : nullptr);
+      // the ring overlays SMEM last written by ordinary stores: order those before the
+      // bulk copies
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const int cs = gate ? a.cs_g : a.cs_u, np = gate ? a.Gg : G - a.Gg;
+      const PhaseWork wk{d, min(d, rank * cs), min(d, (rank + 1) * cs), min(d, np * cs), np, a.wmin_b,
+                         a.ctr + (gate ? 0 : 1)};
+      const bool ok = produce(R, a.S_b, row_bytes, row_bytes, 1, reinterpret_cast<const char*>(gate ? a.wt_gate : a.wt_up),
+                              wk, flags, ps, pol, b == 0 ? a.trace : nullptr);
       if (!ok && (threadIdx.x & 31) == 0) s_abort = 1;
     } else {
-      if (!consume_store<BF16>(R, a.S_b, row_bytes, ffn, full_par, gate ? acc_g : acc_u,
-                               b == 0 ? a.trace : nullptr))
+      if (!consume<BF16>(R, a.S_b, row_bytes, row_bytes, ffn, full_par, vals, gate ? acc_g : acc_u,
+                         b == 0 ? a.trace : nullptr))
         s_abort = 1;
     }
   }
@@ -501,61 +589,75 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   }
   stamp(a.stamps, 2);
   cta_time(a.cta_t, 1);
-  if (!grid_sync_fixed(a.bar, G, a.status)) return;
+  // the ring is drained: fetch c_down into the staging buffer while waiting for the grid
+  if (threadIdx.x == 0 && a.mode == WINA_GATE_TOPK) {
+    mbar_expect_tx(aux, (uint32_t)ffn * 4u);
+    bulk_copy_g2s(stage_in, a.c_down, (uint32_t)ffn * 4u, aux, pol);
+  }
+  if (!grid_sync_fixed(a.bar, G, a.status)) {
+    if (threadIdx.x == 0 && a.mode == WINA_GATE_TOPK) {  // let the issued copy land before exiting
+      mbar_arrive(aux);
+      mbar_wait(aux, 1u);
+    }
+    return;
+  }
   stamp(a.stamps, 3);
 
   // ---------------- C/D: h for every channel, the down scores, the down bitmask ----------------
+  touch_pages(a.wt_down, (size_t)d * ffn * ESZ);  // as in phase A, for the down rows
   if (b == 0 && threadIdx.x == 0) {
     a.ctr[0] = 0u;  // every CTA is past phase B: the gate/up unit counters can be reset
     a.ctr[1] = 0u;
   }
   {
-    constexpr int U = 3;  // float4 columns per thread per round, all loads issued first
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    const int m4 = ffn / 4;
+    // g into vals, u into keys (bulk copies); h replaces g and the score replaces u in
+    // place; the score histogram is filled on the way
     const bool topk = a.mode == WINA_GATE_TOPK;
-    for (int q0 = threadIdx.x; q0 < m4; q0 += U * kFT) {
-      float4 g4[U], u4[U], c4[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int q = q0 + u * kFT;
-        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        g4[u] = q < m4 ? __ldcg(reinterpret_cast<const float4*>(acc_g) + q) : z;
-        u4[u] = q < m4 ? __ldcg(reinterpret_cast<const float4*>(acc_u) + q) : z;
-        c4[u] = (q < m4 && topk) ? __ldg(reinterpret_cast<const float4*>(a.c_down) + q) : z;
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int q = q0 + u * kFT;
-        if (q >= m4) continue;
-        float4 h4;
-        h4.x = silu_f(g4[u].x) * u4[u].x;
-        h4.y = silu_f(g4[u].y) * u4[u].y;
-        h4.z = silu_f(g4[u].z) * u4[u].z;
-        h4.w = silu_f(g4[u].w) * u4[u].w;
-        reinterpret_cast<float4*>(vals)[q] = h4;
-        if (b == G - 1) reinterpret_cast<float4*>(a.h)[q] = h4;
-        if (topk) {
-          uint4 k4;
-          k4.x = __float_as_uint(fabsf(h4.x * c4[u].x));
-          k4.y = __float_as_uint(fabsf(h4.y * c4[u].y));
-          k4.z = __float_as_uint(fabsf(h4.z * c4[u].z));
-          k4.w = __float_as_uint(fabsf(h4.w * c4[u].w));
-          reinterpret_cast<uint4*>(keys)[q] = k4;
-          kmin = min(min(kmin, min(k4.x, k4.y)), min(k4.z, k4.w));
-          kmax = max(max(kmax, max(k4.x, k4.y)), max(k4.z, k4.w));
-        }
+    if (threadIdx.x == 0) {
+      // the sums were made by other SMs' atomics (generic proxy); order them before the
+      // bulk copies (async proxy) that read them
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      mbar_arrive_expect_tx(aux, 2u * (uint32_t)ffn * 4u);
+      bulk_copy_g2s(vals, acc_g, (uint32_t)ffn * 4u, aux, pol);
+      bulk_copy_g2s(keys, acc_u, (uint32_t)ffn * 4u, aux, pol);
+    }
+    for (int i = threadIdx.x; i < kSelBins; i += kFT) hist[i] = 0u;
+    if (!mbar_wait(aux, 1u)) s_abort = 1;
+    __syncthreads();
+    if (s_abort) {
+      record_status(a.status, WINA_ERR_TIMEOUT);
+      return;
+    }
+    const float* cdn = reinterpret_cast<const float*>(stage_in);
+    for (int q = threadIdx.x; q < ffn / 4; q += kFT) {
+      const float4 g4 = reinterpret_cast<const float4*>(vals)[q];
+      const float4 u4 = reinterpret_cast<const float4*>(keys)[q];
+      float4 h4;
+      h4.x = silu_f(g4.x) * u4.x;
+      h4.y = silu_f(g4.y) * u4.y;
+      h4.z = silu_f(g4.z) * u4.z;
+      h4.w = silu_f(g4.w) * u4.w;
+      reinterpret_cast<float4*>(vals)[q] = h4;
+      if (b == G - 1) reinterpret_cast<float4*>(a.h)[q] = h4;
+      if (topk) {
+        const float4 c4 = reinterpret_cast<const float4*>(cdn)[q];
+        uint4 k4;
+        k4.x = __float_as_uint(fabsf(h4.x * c4.x));
+        k4.y = __float_as_uint(fabsf(h4.y * c4.y));
+        k4.z = __float_as_uint(fabsf(h4.z * c4.z));
+        k4.w = __float_as_uint(fabsf(h4.w * c4.w));
+        reinterpret_cast<uint4*>(keys)[q] = k4;
+        atomicAdd(&hist[k4.x >> 19], 1u);
+        atomicAdd(&hist[k4.y >> 19], 1u);
+        atomicAdd(&hist[k4.z >> 19], 1u);
+        atomicAdd(&hist[k4.w >> 19], 1u);
       }
     }
     stamp(a.stamps, 4);
-    if (a.mode == WINA_GATE_TOPK) {
-      uint32_t mn, mx;
-      block_minmax_u32<kFT>(kmin, kmax, red, mn, mx);
-      stamp(a.stamps, 11);
-      select_topk_flags<kFT>(keys, ffn, a.k_down, mn, mx, hist, cand, red, flags);
+    if (topk) {
+      select_topk_flags_radix<kFT>(keys, ffn, a.k_down, hist, cand, red, flags, b == 0 ? a.stamps + 14 : nullptr);
     } else {
       __syncthreads();
-      stamp(a.stamps, 11);
       if (a.mode == WINA_GATE_STAT)
         flags_from_threshold(vals, ffn, spark_threshold(vals, ffn, a.z, dred), flags);
       else
@@ -564,21 +666,29 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   }
   __syncthreads();
   stamp(a.stamps, 5);
-  stamp(a.stamps, 12);
   if (b == G - 1) write_keep_bytes(flags, ffn, a.keep_d);
   stamp(a.stamps, 6);
   cta_time(a.cta_t, 2);
 
   // ---------------- E: stream kept down rows through the ring ----------------
   {
-    const uint32_t row_bytes = (uint32_t)d * ESZ;
+    // the down scores are no longer needed: the ring now starts at keys
+    const uint32_t row_bytes = (uint32_t)d * ESZ, stage_bytes = (uint32_t)a.rows_e * row_bytes;
+    const int S = min(kMaxStages, (int)(((uint32_t)a.smem - SL.keys) / stage_bytes));
+    Ring RE = R;
+    RE.base = reinterpret_cast<char*>(smraw + SL.keys);
     if (producer) {
-      const bool ok = produce(R, a.S_e, row_bytes, reinterpret_cast<const char*>(a.wt_down), ffn, a.uw_e, a.ctr + 2,
-                              flags, vals, ps, pol, b == 0 ? a.trace + 128 : nullptr);
-      if (!ok && (threadIdx.x & 31) == 0) s_abort = 1;
-    } else {
-      if (!consume_store<BF16>(R, a.S_e, row_bytes, d, full_par, a.acc_y, b == 0 ? a.trace + 128 : nullptr))
+      // the ring overlays SMEM last written by ordinary stores: order those before the
+      // bulk copies
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const PhaseWork wk{ffn, min(ffn, b * a.cs_e), min(ffn, (b + 1) * a.cs_e), min(ffn, G * a.cs_e), G, a.wmin_e,
+                         a.ctr + 2};
+      if (!produce(RE, S, row_bytes, stage_bytes, a.rows_e, reinterpret_cast<const char*>(a.wt_down), wk, flags, ps,
+                   pol) &&
+          (threadIdx.x & 31) == 0)
         s_abort = 1;
+    } else {
+      if (!consume<BF16>(RE, S, row_bytes, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
     }
   }
   __syncthreads();
@@ -679,14 +789,17 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
     const uint32_t esz = bf16 ? 2u : 4u;
     const SmemLayout SLay = ffn_smem_layout((int)d, (int)ffn);
     size_t ring = SLay.ring < kMaxSmem ? (kMaxSmem - SLay.ring) / 128 * 128 : 0;
-    if (ring < kMinRing) ring = 0;
-    const uint32_t rb_b = (uint32_t)ffn * esz, rb_e = (uint32_t)d * esz;
+    if (ring < ffn_min_ring((int)d, (int)ffn)) ring = 0;
+    const uint32_t rb_b = (uint32_t)ffn * esz;
     const int S_b = (int)std::min<size_t>(kMaxStages, ring / rb_b);
-    const int S_e = (int)std::min<size_t>(kMaxStages, ring / rb_e);
     const size_t smem = kMaxSmem;
     const int G = bf16 ? max_coresident_grid(k_ffn_fused<true>, kFT, smem)
                        : max_coresident_grid(k_ffn_fused<false>, kFT, smem);
-    if (G >= 2 && S_b >= 2 && S_e >= 2) {
+    // phase E: rows per stage (pieces of up to that many adjacent rows per bulk copy),
+    // at least two stages in the ring, which then starts at keys
+    const uint32_t rb_e = (uint32_t)d * esz;
+    const int rows_e = SLay.keys < kMaxSmem ? (int)std::min<size_t>(4, (kMaxSmem - SLay.keys) / (2 * (size_t)rb_e)) : 0;
+    if (G >= 2 && S_b >= 2 && rows_e >= 1) {
       FfnParams p;
       p.wt_gate = f->wt_gate;
       p.wt_up = f->wt_up;
@@ -710,22 +823,24 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
         Gg = (int)((G * k_gate + (k_gate + k_up) / 2) / (k_gate + k_up));
       Gg = std::max(1, std::min(G - 1, Gg));
       p.Gg = Gg;
-      // channels per work unit: enough to hold ~64 KB of kept rows (at least 4 rows),
-      // so that a unit's copies are issued by several lanes at once
-      auto unit_width = [](int64_t n, int64_t kept, uint32_t row_bytes) {
-        const double keep = kept > 0 ? (double)kept / (double)n : 1.0;
-        const double rows = std::max(4.0, 65536.0 / row_bytes);
-        const int w = (int)std::ceil(rows / keep);
-        int p2 = 1;
-        while (p2 < w && p2 < 32) p2 *= 2;
-        return p2;
-      };
+      // each CTA first streams its own block of channels (no counter round trip at the
+      // start); the counters hand out the rest in guided units, the shortest about one
+      // row (gate/up) or two rows (down)
+      constexpr double kOwnShare = 0.7;
+      p.cs_g = (int)(kOwnShare * (double)d / (double)Gg);
+      p.cs_u = (int)(kOwnShare * (double)d / (double)(G - Gg));
+      p.cs_e = (int)(kOwnShare * (double)ffn / (double)G);
       const int64_t kept_b = mode == WINA_GATE_TOPK ? std::max(k_gate, k_up) : (mode == WINA_GATE_DENSE ? d : (int64_t)(s * d));
       const int64_t kept_e = mode == WINA_GATE_TOPK ? k_down : (mode == WINA_GATE_DENSE ? ffn : (int64_t)(s * ffn));
-      p.uw_b = unit_width(d, kept_b, rb_b);
-      p.uw_e = unit_width(ffn, kept_e, rb_e);
+      auto min_width = [](int64_t n, int64_t kept, double rows) {
+        const double keep = kept > 0 ? std::min(1.0, (double)kept / (double)n) : 1.0;
+        return (int)std::max(1.0, std::min(32.0, std::ceil(rows / keep)));
+      };
+      p.wmin_b = min_width(d, kept_b, 1.0);
+      p.wmin_e = min_width(ffn, kept_e, 2.0);
       p.S_b = S_b;
-      p.S_e = S_e;
+      p.rows_e = rows_e;
+      p.smem = (int)smem;
       p.bar = reinterpret_cast<GridBarrier*>(w + L.bar);
       p.ctr = reinterpret_cast<unsigned*>(w + L.ctr);
       p.h = reinterpret_cast<float*>(w + L.h);

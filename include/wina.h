@@ -106,10 +106,13 @@ typedef struct {
  *   keep_up   uint8   [batch][d]    1 where the up projection's input channel was kept
  *   keep_down uint8   [batch][ffn]  1 where the down projection's input channel was kept
  *   stamps    int64   [16]          single-token kernel only: SM clock (clock64) of CTA 0
- *                                   at its phase boundaries: 0 start, 1 gate/up kept sets
- *                                   known, 2 gate/up rows streamed, 3 barrier, 4 h written,
- *                                   5 barrier, 6 down kept set known, 7 down rows
- *                                   streamed, 8 barrier, 9 end
+ *                                   at its phase boundaries: 0 start, 10 x and c landed,
+ *                                   11 gate/up scores made, 12 boundary bin found,
+ *                                   13 channels outside it flagged, 1 gate/up kept sets
+ *                                   known, 2 gate/up rows streamed, 3 grid barrier passed,
+ *                                   4 h and down scores made, 14 / 15 as 12 / 13 for down,
+ *                                   5 down kept set known, 6 its bytes written, 7 down
+ *                                   rows streamed, 8 / 9 end
  *   cta_t     uint64  [CTAs][4]     single-token kernel only: global timer (ns) at which
  *                                   each CTA finished phases 1, 2, 6 and 7 above        */
 typedef struct {
