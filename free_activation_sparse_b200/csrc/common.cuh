@@ -103,214 +103,6 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* red, u
 // exact top-K selection on non-negative float32 keys
 // ------------------------------------------------------------------------------------
 
-// A selection over keys: channel i is kept iff
-//     (key_i & mask) >  prefix                                  (strictly above), or
-//     (key_i & mask) == prefix and its rank among such i < r      (boundary, by index).
-// neq counts the boundary channels; when r == neq every boundary channel is kept.
-// K = n is {0, 0, n, n}; K = 0 is {0, 0, 0, n}.
-struct Selection {
-  uint32_t mask, prefix, r, neq;
-};
-
-// Radix select of the K-th largest key over NSEL key arrays at once (each of length
-// n in SMEM, with its own K in [1, n)). Digits of 8, 8, 8 and 7 bits are taken from
-// bit 30 down (bit 31 of a non-negative float is 0). A pass histograms the digit of the
-// keys that still match the fixed prefix (SMEM atomics; two histogram buffers, the next
-// one cleared during the current pass), then warp q scans array q's 256 bins from the
-// top (8 per lane, one shuffle scan) and fixes the digit holding the K-th key. Two
-// block barriers per pass. A search ends early once that bin holds exactly the count
-// still needed. `hist` is SMEM of 2 * NSEL * 256 words; NSEL <= NT / 32. Every thread
-// of the block must call it.
-template <int NT, int NSEL>
-__device__ void radix_select(const uint32_t* const (&keys)[NSEL], int n, const int (&K)[NSEL], uint32_t* hist,
-                             Selection (&out)[NSEL]) {
-  __shared__ uint32_t s_res[NSEL][3];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t mask[NSEL], prefix[NSEL], rem[NSEL], neq[NSEL];
-  bool done[NSEL];
-#pragma unroll
-  for (int q = 0; q < NSEL; ++q) {
-    mask[q] = 0u;
-    prefix[q] = 0u;
-    rem[q] = (uint32_t)K[q];
-    neq[q] = (uint32_t)n;
-    done[q] = false;
-  }
-  for (int i = threadIdx.x; i < NSEL * 256; i += NT) hist[i] = 0u;
-  __syncthreads();
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int sh = pass < 3 ? 23 - 8 * pass : 0;
-    const uint32_t dm = pass < 3 ? 0xffu : 0x7fu;
-    uint32_t* H = hist + (pass & 1) * NSEL * 256;
-    uint32_t* Hn = hist + ((pass & 1) ^ 1) * NSEL * 256;
-    for (int i = threadIdx.x; i < n; i += NT) {
-#pragma unroll
-      for (int q = 0; q < NSEL; ++q) {
-        if (done[q]) continue;  // uniform across the block
-        const uint32_t k = keys[q][i];
-        if ((k & mask[q]) == prefix[q]) atomicAdd(&H[q * 256 + ((k >> sh) & dm)], 1u);
-      }
-    }
-    for (int i = threadIdx.x; i < NSEL * 256; i += NT) Hn[i] = 0u;
-    __syncthreads();
-    if (warp < NSEL) {
-      const int q = warp;
-      if (!done[q]) {
-        uint32_t c[8];
-        uint32_t local = 0u;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          c[j] = H[q * 256 + 255 - (lane * 8 + j)];  // descending bins
-          local += c[j];
-        }
-        uint32_t incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        const uint32_t above = incl - local;
-        if (above < rem[q] && incl >= rem[q]) {  // exactly one lane holds the crossing
-          uint32_t cum = above;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (cum + c[j] >= rem[q]) {
-              s_res[q][0] = 255u - (uint32_t)(lane * 8 + j);
-              s_res[q][1] = rem[q] - cum;
-              s_res[q][2] = c[j];
-              break;
-            }
-            cum += c[j];
-          }
-        }
-      }
-    }
-    __syncthreads();
-    bool all_done = true;
-#pragma unroll
-    for (int q = 0; q < NSEL; ++q) {
-      if (done[q]) continue;
-      rem[q] = s_res[q][1];
-      neq[q] = s_res[q][2];
-      prefix[q] |= s_res[q][0] << sh;
-      mask[q] |= dm << sh;
-      if (neq[q] == rem[q] || pass == 3) done[q] = true;
-      all_done = all_done && done[q];
-    }
-    if (all_done) break;
-    // s_res is rewritten only after the next pass's first barrier; H (this pass's
-    // buffer) is cleared by the next pass before its barrier, after everyone has
-    // passed the barrier above that ended the reads of it.
-  }
-#pragma unroll
-  for (int q = 0; q < NSEL; ++q) out[q] = Selection{mask[q], prefix[q], rem[q], neq[q]};
-  __syncthreads();
-}
-
-// Top-K of NSEL key arrays of length n (K = 0 and K >= n handled without a search).
-// `hist`: SMEM of 2 * NSEL * 256 words.
-template <int NT, int NSEL>
-__device__ __forceinline__ void select_topk_multi(const uint32_t* const (&keys)[NSEL], int n, const int (&K)[NSEL],
-                                                  uint32_t* hist, Selection (&out)[NSEL]) {
-  int Ks[NSEL];
-  bool search = false;
-#pragma unroll
-  for (int q = 0; q < NSEL; ++q) {
-    Ks[q] = K[q] <= 0 ? 0 : (K[q] >= n ? n : K[q]);
-    search = search || (Ks[q] > 0 && Ks[q] < n);
-  }
-  if (search) {
-    // arrays that need no search still run through the passes with K = 1 and are
-    // overwritten below; this keeps the block's control flow uniform
-    int Kr[NSEL];
-#pragma unroll
-    for (int q = 0; q < NSEL; ++q) Kr[q] = (Ks[q] > 0 && Ks[q] < n) ? Ks[q] : 1;
-    radix_select<NT, NSEL>(keys, n, Kr, hist, out);
-  }
-#pragma unroll
-  for (int q = 0; q < NSEL; ++q) {
-    if (Ks[q] == 0) out[q] = Selection{0u, 0u, 0u, (uint32_t)n};
-    if (Ks[q] == n) out[q] = Selection{0u, 0u, (uint32_t)n, (uint32_t)n};
-  }
-}
-
-template <int NT>
-__device__ __forceinline__ Selection select_topk_block(const uint32_t* keys, int n, int K, uint32_t* hist) {
-  const uint32_t* ks[1] = {keys};
-  const int kk[1] = {K};
-  Selection out[1];
-  select_topk_multi<NT, 1>(ks, n, kk, hist, out);
-  return out[0];
-}
-
-// Warp-ballot compaction of a Selection, in ascending index order. Warp w walks the
-// contiguous segment [w*seg, (w+1)*seg) 32 channels at a time; a first walk counts the
-// strictly-above and boundary channels per warp, a scan over warps gives each warp its
-// bases, and a second walk computes every kept channel's output position
-//     pos(i) = #strict before i + min(#boundary before i, r).
-// emit(i, pos) is called for kept channels with lo <= pos < hi. `wsm` is SMEM of
-// >= 2*NT/32 words. Every thread of the block must call it.
-template <int NT, typename Emit>
-__device__ void compact_selection(const uint32_t* keys, int n, Selection sel, uint32_t lo, uint32_t hi, uint32_t* wsm,
-                                  Emit emit) {
-  constexpr int NW = NT / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int seg = (((n + NW - 1) / NW) + 31) & ~31;
-  const int b0 = warp * seg;
-  const int b1 = min(n, b0 + seg);
-  uint32_t cs = 0, ce = 0;
-  for (int base = b0; base < b1; base += 32) {
-    const int i = base + lane;
-    const bool in = i < b1;
-    const uint32_t mk = in ? (keys[i] & sel.mask) : 0u;
-    cs += __popc(__ballot_sync(0xffffffffu, in && mk > sel.prefix));
-    ce += __popc(__ballot_sync(0xffffffffu, in && mk == sel.prefix));
-  }
-  if (lane == 0) {
-    wsm[warp] = cs;
-    wsm[NW + warp] = ce;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t a = lane < NW ? wsm[lane] : 0u;
-    const uint32_t e = lane < NW ? wsm[NW + lane] : 0u;
-    uint32_t ia = a, ie = e;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t ya = __shfl_up_sync(0xffffffffu, ia, o);
-      const uint32_t ye = __shfl_up_sync(0xffffffffu, ie, o);
-      if (lane >= o) {
-        ia += ya;
-        ie += ye;
-      }
-    }
-    if (lane < NW) {
-      wsm[lane] = ia - a;
-      wsm[NW + lane] = ie - e;
-    }
-  }
-  __syncthreads();
-  uint32_t sbase = wsm[warp], ebase = wsm[NW + warp];
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int base = b0; base < b1; base += 32) {
-    const int i = base + lane;
-    const bool in = i < b1;
-    const uint32_t mk = in ? (keys[i] & sel.mask) : 0u;
-    const bool st = in && mk > sel.prefix;
-    const bool eq = in && mk == sel.prefix;
-    const uint32_t sb = __ballot_sync(0xffffffffu, st);
-    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-    const uint32_t erank = ebase + __popc(eb & lt);
-    const bool keep = st || (eq && erank < sel.r);
-    const uint32_t pos = sbase + __popc(sb & lt) + min(erank, sel.r);
-    if (keep && pos >= lo && pos < hi) emit(i, pos);
-    sbase += __popc(sb);
-    ebase += __popc(eb);
-  }
-  __syncthreads();  // wsm may be reused right after
-}
-
 // Ballot compaction of a predicate (ascending index order): first counts, then calls
 // range(total, &lo, &hi) on every thread to choose the window of positions wanted, then
 // emit(i, pos) for kept channels with lo <= pos < hi. Returns the total kept count.
@@ -613,95 +405,6 @@ __device__ void hist_crossing(const uint32_t* __restrict__ hist, uint32_t r, uin
   *cnt = s_cnt;
 }
 
-// The candidates cand[0..nc) = (key, index) pairs: set the flag bits of the r with the
-// highest (key desc, index asc). Warp w ranks candidates w, w + NT/32, ...: its lanes
-// compare that candidate with a 32-strided slice of the others each and sum the counts.
-// Ends with a block barrier.
-template <int NT>
-__device__ __forceinline__ void rank_and_keep(const uint32_t* __restrict__ cand, int nc, uint32_t r,
-                                              uint32_t* __restrict__ flags) {
-  constexpr int NW = NT / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int c = warp; c < nc; c += NW) {
-    const uint32_t kc = cand[2 * c], ic = cand[2 * c + 1];
-    uint32_t above = 0u;
-    for (int o = lane; o < nc; o += 32) {
-      const uint32_t ko = cand[2 * o], io = cand[2 * o + 1];
-      above += (ko > kc || (ko == kc && io < ic)) ? 1u : 0u;
-    }
-    above = __reduce_add_sync(0xffffffffu, above);
-    if (lane == 0 && above < r) atomicOr(&flags[ic >> 5], 1u << (ic & 31));
-  }
-  __syncthreads();
-}
-
-// Kept-channel bitmask of the exact top-K of keys[0..n) in SMEM (ties to the lower
-// index), given the keys' min and max. One histogram pass over a linear map of the key
-// bits onto kSelBins bins (monotone, so bins are ordered like the keys), a two-level
-// scan for the bin holding the K-th key, then one pass that sets the flags of every
-// channel outside that bin and gathers the bin's keys; those are ranked exactly and
-// the kept ones set. If the bin holds more than kSelCand keys, the general search
-// (select_threshold) decides. flags[w] bit l = channel 32w + l is kept.
-// SMEM: hist [kSelBins], cand [2 * kSelCand], red [>= 2 * NT/32 + 8]. All threads call.
-template <int NT>
-__device__ void select_topk_flags(const uint32_t* __restrict__ keys, int n, int K, uint32_t mn, uint32_t mx,
-                                  uint32_t* __restrict__ hist, uint32_t* __restrict__ cand, uint32_t* __restrict__ red,
-                                  uint32_t* __restrict__ flags) {
-  constexpr int NW = NT / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = (n + 31) / 32;
-  __shared__ uint32_t s_ncand;
-  if (K <= 0 || K >= n || mn == mx) {
-    // nothing, everything, or all keys equal (then the first K by index)
-    const int keep = K <= 0 ? 0 : (K >= n ? n : K);
-    for (int w = threadIdx.x; w < nw; w += NT) {
-      const int rem = keep - w * 32;
-      flags[w] = rem >= 32 ? 0xffffffffu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
-    }
-    __syncthreads();
-    return;
-  }
-  const float scale = (float)kSelBins / ((float)(mx - mn) + 1.0f);
-  auto bin_of = [&](uint32_t k) { return min(kSelBins - 1, (int)((float)(k - mn) * scale)); };
-  for (int i = threadIdx.x; i < kSelBins; i += NT) hist[i] = 0u;
-  if (threadIdx.x == 0) s_ncand = 0u;
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += NT) atomicAdd(&hist[bin_of(keys[i])], 1u);
-  __syncthreads();
-  int B;
-  uint32_t above, cnt;
-  hist_crossing<NT>(hist, (uint32_t)K, red, &B, &above, &cnt);
-  if (cnt > (uint32_t)kSelCand) {
-    const Threshold t = select_threshold<NT>(keys, n, K, hist, cand, red);
-    for (int w = warp; w < nw; w += NW) {
-      const int j = w * 32 + lane;
-      const uint32_t bits = __ballot_sync(0xffffffffu, j < n && kept_by(t, keys[j], j));
-      if (lane == 0) flags[w] = bits;
-    }
-    __syncthreads();
-    return;
-  }
-  const uint32_t r = (uint32_t)K - above;  // kept among the bin's keys
-  for (int w = warp; w < nw; w += NW) {
-    const int j = w * 32 + lane;
-    int bj = -1;
-    uint32_t k = 0u;
-    if (j < n) {
-      k = keys[j];
-      bj = bin_of(k);
-    }
-    const uint32_t bits = __ballot_sync(0xffffffffu, bj > B);
-    if (lane == 0) flags[w] = bits;
-    if (bj == B) {
-      const uint32_t at = atomicAdd(&s_ncand, 1u);
-      cand[2 * at] = k;
-      cand[2 * at + 1] = (uint32_t)j;
-    }
-  }
-  __syncthreads();
-  rank_and_keep<NT>(cand, (int)s_ncand, r, flags);
-}
-
 // Kept-channel bitmask of the exact top-K of keys[0..n) in SMEM (ties to the lower
 // index), given hist = the counts of the keys' top 12 bits (key >> 19; bit 31 of a
 // non-negative float is 0), which the caller fills while it produces the keys. A
@@ -709,9 +412,9 @@ __device__ void select_topk_flags(const uint32_t* __restrict__ keys, int n, int 
 // channel outside that bin and gathers the bin's keys, which are ranked exactly. If the
 // bin holds more than kSelCand keys, the general search (select_threshold) decides.
 // flags[w] bit l = channel 32w + l is kept. SMEM: keys 16-byte aligned and readable
-// up to the next multiple of 128 entries (the excess is ignored), hist [kSelBins]
-// (filled), cand [2 * kSelCand], red [>= 2 * NT/32 + 8]. Every thread of the block
-// must call it.
+// up to the next multiple of 128 entries (the excess is ignored), hist [kSelBins + 256]
+// (the first kSelBins filled, the last 256 zero), cand [2 * kSelCand], red
+// [>= 2 * NT/32 + 8]. Every thread of the block must call it.
 template <int NT>
 __device__ void select_topk_flags_radix(const uint32_t* __restrict__ keys, int n, int K, uint32_t* __restrict__ hist,
                                         uint32_t* __restrict__ cand, uint32_t* __restrict__ red,
@@ -720,7 +423,6 @@ __device__ void select_topk_flags_radix(const uint32_t* __restrict__ keys, int n
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nw = (n + 31) / 32;
-  __shared__ uint32_t s_ncand;
   if (K <= 0 || K >= n) {
     const int keep = K <= 0 ? 0 : n;
     for (int w = threadIdx.x; w < nw; w += NT) {
@@ -730,7 +432,6 @@ __device__ void select_topk_flags_radix(const uint32_t* __restrict__ keys, int n
     __syncthreads();
     return;
   }
-  if (threadIdx.x == 0) s_ncand = 0u;
   __syncthreads();  // the caller's histogram updates are complete
   int B;
   uint32_t above, cnt;
@@ -747,46 +448,122 @@ __device__ void select_topk_flags_radix(const uint32_t* __restrict__ keys, int n
     return;
   }
   const uint32_t r = (uint32_t)K - above;  // kept among the bin's keys
-  // flags outside the boundary bin, and the bin's keys gathered: each lane takes four
-  // consecutive channels (one 16-byte load), so a warp covers four flag words per step;
-  // eight lanes' nibbles are merged into a word by shuffles
+  // 1. one pass over the keys: flags of the channels above the boundary bin B; the bin's
+  //    keys go to per-warp lists (in the first-level histogram's place, no longer
+  //    needed) and into a 256-bin histogram of their next 8 bits (`sub`, zeroed by the
+  //    caller). Each lane takes four consecutive channels (one 16-byte load); eight
+  //    lanes' nibbles are merged into a flag word by shuffles.
+  constexpr int kSlab = 64;  // list entries per warp
+  uint32_t* slab = hist + (size_t)warp * kSlab * 2;
+  uint32_t* sub = hist + kSelBins;
+  uint32_t nmine = 0u;  // this warp's list length (uniform in the warp)
   const int n128 = (n + 127) / 128;
   for (int q = warp; q < n128; q += NW) {
     const int j0 = q * 128 + lane * 4;
     const uint4 k4 = reinterpret_cast<const uint4*>(keys)[q * 32 + lane];
     const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
-    uint32_t nib = 0u, inb[4];
+    uint32_t above_nib = 0u, inb[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const bool in = j0 + e < n;
-      const int bj = (int)(kk[e] >> 19);
-      nib |= (in && bj > B) ? (1u << e) : 0u;
-      inb[e] = __ballot_sync(0xffffffffu, in && bj == B);
+      const int bj = j0 + e < n ? (int)(kk[e] >> 19) : -1;
+      above_nib |= bj > B ? (1u << e) : 0u;
+      inb[e] = __ballot_sync(0xffffffffu, bj == B);
     }
-    uint32_t v = nib << (4 * (lane & 7));
-    v |= __shfl_xor_sync(0xffffffffu, v, 1);
-    v |= __shfl_xor_sync(0xffffffffu, v, 2);
-    v |= __shfl_xor_sync(0xffffffffu, v, 4);
-    if ((lane & 7) == 0 && q * 4 + (lane >> 3) < nw) flags[q * 4 + (lane >> 3)] = v;
+    uint32_t fa = above_nib << (4 * (lane & 7));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) fa |= __shfl_xor_sync(0xffffffffu, fa, o);
+    const int w = q * 4 + (lane >> 3);
+    if ((lane & 7) == 0 && w < nw) flags[w] = fa;
     const uint32_t tot = __popc(inb[0]) + __popc(inb[1]) + __popc(inb[2]) + __popc(inb[3]);
     if (tot) {  // uniform across the warp
       const uint32_t lt = (1u << lane) - 1u;
-      uint32_t base = 0u;
-      if (lane == 0) base = atomicAdd(&s_ncand, tot);
-      base = __shfl_sync(0xffffffffu, base, 0) + __popc(inb[0] & lt) + __popc(inb[1] & lt) + __popc(inb[2] & lt) +
-             __popc(inb[3] & lt);
+      uint32_t at = nmine + __popc(inb[0] & lt) + __popc(inb[1] & lt) + __popc(inb[2] & lt) + __popc(inb[3] & lt);
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if ((inb[e] >> lane) & 1u) {
-          cand[2 * base] = kk[e];
-          cand[2 * base + 1] = (uint32_t)(j0 + e);
-          ++base;
+          if (at < (uint32_t)kSlab) {
+            slab[2 * at] = kk[e];
+            slab[2 * at + 1] = (uint32_t)(j0 + e);
+          }
+          atomicAdd(&sub[(kk[e] >> 11) & 255u], 1u);
+          ++at;
         }
+      nmine += tot;
     }
+  }
+  __shared__ uint32_t s_len[NT / 32], s_b2, s_above2, s_nties, s_over;
+  if (lane == 0) s_len[warp] = nmine;
+  if (threadIdx.x == 0) {
+    s_nties = 0u;
+    s_over = 0u;
   }
   __syncthreads();
   if (st && threadIdx.x == 0) st[1] = clock64();
-  rank_and_keep<NT>(cand, (int)s_ncand, r, flags);
+  // 2. warp 0 finds the sub-bin B2 holding the r-th largest of the bin's keys
+  if (warp == 0) {
+    uint32_t v[8], t = 0u;  // lane l: sub-bins 255 - 8l, ..., 248 - 8l (from the top)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      v[e] = sub[255 - 8 * lane - e];
+      t += v[e];
+    }
+    uint32_t x = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    uint32_t ab = x - t;  // keys in sub-bins above this lane's
+    const bool hit = ab < r && ab + t >= r;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (hit && ab < r && ab + v[e] >= r) {
+        s_b2 = (uint32_t)(255 - 8 * lane - e);
+        s_above2 = ab;
+      }
+      ab += v[e];
+    }
+    bool over = false;
+    for (int w2 = lane; w2 < NW; w2 += 32) over |= s_len[w2] > (uint32_t)kSlab;
+    if (__any_sync(0xffffffffu, over) && lane == 0) s_over = 1u;
+  }
+  __syncthreads();
+  if (s_over) {
+    // a warp's list overflowed (keys bunched in the bin): the general search decides
+    const Threshold t = select_threshold<NT>(keys, n, K, hist, cand, red);
+    for (int w = warp; w < nw; w += NW) {
+      const int j = w * 32 + lane;
+      const uint32_t bits = __ballot_sync(0xffffffffu, j < n && kept_by(t, keys[j], j));
+      if (lane == 0) flags[w] = bits;
+    }
+    __syncthreads();
+    return;
+  }
+  // 3. keys above B2 are kept; those in B2 go to a short list
+  const uint32_t B2 = s_b2, r2 = r - s_above2;
+  for (uint32_t e = lane; e < nmine; e += 32) {
+    const uint32_t k = slab[2 * e], ch = slab[2 * e + 1], sb = (k >> 11) & 255u;
+    if (sb > B2) {
+      atomicOr(&flags[ch >> 5], 1u << (ch & 31));
+    } else if (sb == B2) {
+      const uint32_t at = atomicAdd(&s_nties, 1u);
+      cand[2 * at] = k;
+      cand[2 * at + 1] = ch;
+    }
+  }
+  __syncthreads();
+  // 4. the r2 highest of that list (ties to the lower channel) are kept
+  const uint32_t nt = s_nties;
+  for (uint32_t c = threadIdx.x; c < nt; c += NT) {
+    const uint32_t kc = cand[2 * c], ic = cand[2 * c + 1];
+    uint32_t a = 0u;
+    for (uint32_t o = 0; o < nt; ++o) {
+      const uint32_t ko = cand[2 * o], io = cand[2 * o + 1];
+      a += (ko > kc || (ko == kc && io < ic)) ? 1u : 0u;
+    }
+    if (a < r2) atomicOr(&flags[ic >> 5], 1u << (ic & 31));
+  }
+  __syncthreads();
 }
 
 // ------------------------------------------------------------------------------------

@@ -141,18 +141,6 @@ __device__ __forceinline__ void cta_time(unsigned long long* t, int i) {
 // kept-channel bitmask
 // ------------------------------------------------------------------------------------
 
-// flags[w] bit l = channel 32w + l is kept by the top-K threshold.
-__device__ void flags_from_topk(const uint32_t* keys, int n, const Threshold& t, uint32_t* flags) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = (n + 31) / 32;
-  for (int w = warp; w < nw; w += kFT / 32) {
-    const int j = w * 32 + lane;
-    const bool k = j < n && kept_by(t, keys[j], j);
-    const uint32_t bits = __ballot_sync(0xffffffffu, k);
-    if (lane == 0) flags[w] = bits;
-  }
-}
-
 // flags for the Spark threshold: v_j > t (float64 comparison).
 __device__ void flags_from_threshold(const float* v, int n, double t, uint32_t* flags) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -251,10 +239,12 @@ __device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage
     const int len = (after ? __ffs(after) - 1 : 32) - lane;  // rows in the piece headed here
     const int np = __popc(heads), pos = __popc(heads & lt);
     bool ok = true;
-    for (int r0 = 0; r0 < np; r0 += S) {
-      const int nr = min(S, np - r0);
-      // each lane issues its piece as soon as its stage is free (the oldest first), so
-      // the ring is refilled stage by stage rather than a round at a time
+    // rounds of at most half the ring: a round ends when its last stage is free, and
+    // the other half of the ring stays in flight meanwhile
+    const int RS = max(1, S / 2);
+    for (int r0 = 0; r0 < np; r0 += RS) {
+      const int nr = min(RS, np - r0);
+      // each lane issues its piece as soon as its stage is free (the oldest first)
       bool mine = head && pos >= r0 && pos < r0 + nr;
       const int s = (stage + pos - r0) % S;
       const bool was_used = (ps.used >> s) & 1u;
@@ -262,7 +252,7 @@ __device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage
       unsigned long long t0 = 0;
       while (__any_sync(0xffffffffu, mine)) {
         if (!mine) continue;
-        if (!was_used || mbar_try_wait(&R.empty[s], par)) {
+        if (!was_used || mbar_test_wait(&R.empty[s], par)) {
           const uint32_t bytes = (uint32_t)len * row_bytes;
           R.meta_row[s] = j;
           R.meta_cnt[s] = len;
@@ -524,7 +514,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
     // touch every 2 MB page of this projection's weights now, so that the address
     // translations are warm when the rows stream (the first rows land later otherwise)
     touch_pages(gate ? a.wt_gate : a.wt_up, (size_t)d * ffn * ESZ);
-    for (int i = threadIdx.x; i < kSelBins; i += kFT) hist[i] = 0u;
+    for (int i = threadIdx.x; i < kSelBins + 256; i += kFT) hist[i] = 0u;  // and the sub-bin counts
     if (!xbulk)
       for (int i = threadIdx.x; i < d; i += kFT) reinterpret_cast<float*>(stage_in)[i] = load_elem(a.x, a.xdt, i);
     if (!mbar_wait(aux, 0u)) s_abort = 1;
@@ -621,7 +611,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       bulk_copy_g2s(vals, acc_g, (uint32_t)ffn * 4u, aux, pol);
       bulk_copy_g2s(keys, acc_u, (uint32_t)ffn * 4u, aux, pol);
     }
-    for (int i = threadIdx.x; i < kSelBins; i += kFT) hist[i] = 0u;
+    for (int i = threadIdx.x; i < kSelBins + 256; i += kFT) hist[i] = 0u;  // and the sub-bin counts
     if (!mbar_wait(aux, 1u)) s_abort = 1;
     __syncthreads();
     if (s_abort) {
