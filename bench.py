@@ -151,6 +151,20 @@ def oracle_sample(p: float, budget_s: float = 12.0, max_tokens: int = 20) -> dic
 # ------------------------------------------------------------------------------------
 
 
+def reduce_max(v: float, world: int, device: str) -> float:
+    """The maximum of v over the ranks of the default process group (every rank must
+    call it; a single process returns v). Times are taken as the max over ranks."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -204,11 +218,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, "cuda")
 
     # ---- untimed setup: L layers of weights (packed + norms on the GPU), inputs ----
     L = args.layers
