@@ -41,6 +41,7 @@ constexpr int kCW = 16;                  // consumer warps
 constexpr int kCT = kCW * 32;            // consumer threads
 constexpr int kFT = kCT + 32;            // threads per CTA (consumers + one producer warp)
 constexpr int kMaxStages = 16;           // ring stages at most
+constexpr int kMaxVpt = 4;               // 16-byte row vectors per consumer thread at most
 constexpr size_t kMaxSmem = 224 * 1024;  // dynamic SMEM per CTA (227 KB per block on sm_100, less static)
 
 struct FfnParams {
@@ -61,6 +62,7 @@ struct FfnParams {
   int cs_g, cs_u, cs_e;  // channels in each CTA's own block: gate, up (phase B), down (E)
   int wmin_b, wmin_e;    // shortest dynamic unit (channels) in phases B and E
   int rows_e;            // phase E: rows per ring stage (longest contiguous copy)
+  int rows_o;            // the same when phase E overlaps the down selection (smaller ring)
   int smem;              // dynamic SMEM bytes of the launch
   int S_b;            // ring stages in phase B
   GridBarrier* bar;
@@ -104,7 +106,7 @@ __host__ __device__ inline SmemLayout ffn_smem_layout(int d, int ffn) {
   L.flags = take((nb + 31) / 32 * 4, 16);
   L.meta_row = take(kMaxStages * 4, 16);
   L.meta_cnt = take(kMaxStages * 4, 16);
-  L.bars = take((2 * kMaxStages + 1) * 8, 16);
+  L.bars = take((2 * kMaxStages + 2) * 8, 16);
   L.keys = take(nb * 4, 128);
   L.ring = take(0, 128);
   L.hist = L.ring;
@@ -162,9 +164,14 @@ __device__ void flags_all(int n, uint32_t* flags) {
 }
 
 // Byte flags for the workspace's diagnostic view.
-__device__ void write_keep_bytes(const uint32_t* flags, int n, uint8_t* out) {
-  for (int j = threadIdx.x; j < n; j += kFT) out[j] = (uint8_t)((flags[j >> 5] >> (j & 31)) & 1u);
+__device__ void write_keep_bytes(const uint32_t* flags, int n, uint8_t* out, int nthreads) {
+  for (int j = threadIdx.x; j < n; j += nthreads) out[j] = (uint8_t)((flags[j >> 5] >> (j & 31)) & 1u);
 }
+
+// Barrier among the consumer warps only (the producer warp keeps streaming).
+struct ConsumerSync {
+  __device__ void operator()() const { asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory"); }
+};
 
 // Spark threshold of v[0..n) in SMEM: mu + sigma * z, moments in float64.
 __device__ double spark_threshold(const float* v, int n, double z, double* dred) {
@@ -220,23 +227,24 @@ struct PhaseWork {
 // distinct. The next unit is requested when a unit starts, so the counter's round trip
 // overlaps the unit's copies, and none is requested while the CTA's own block is
 // streamed. Returns false on a timeout.
+// The producer's tail: after its own block and units, the rows listed in tail[0..*tail_n)
+// (one row each), once `tail_ready` (an mbarrier) has completed its first phase.
+struct Tail {
+  uint64_t* ready;
+  const int* list;
+  const int* n;
+};
+
+template <typename Kept>
 __device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage_bytes, int rmax,
-                        const char* __restrict__ Wt, const PhaseWork& wk, const uint32_t* flags, ProdState& ps,
-                        uint64_t pol, unsigned long long* trace = nullptr) {
+                        const char* __restrict__ Wt, const PhaseWork& wk, Kept kept, ProdState& ps, uint64_t pol,
+                        unsigned long long* trace = nullptr, Tail tail = Tail{nullptr, nullptr, nullptr}) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u, le = lt | (1u << lane);
   int stage = 0;
-  // kept rows of channels [j0, j1), j1 - j0 <= 32
-  auto issue = [&](int j0, int j1) {
-    const int j = j0 + lane;
-    const bool k = j < j1 && ((flags[j >> 5] >> (j & 31)) & 1u);
-    const uint32_t km = __ballot_sync(0xffffffffu, k);
-    const uint32_t runs = km & ~(km << 1);                 // first lanes of runs of kept channels
-    const int rs = 31 - __clz(runs & le);                  // start of this lane's run (if kept)
-    const bool head = k && ((lane - rs) % rmax == 0);      // first lane of a piece
+  // this lane heads a piece of `len` rows starting at row j (if head); issue them all
+  auto issue_pieces = [&](bool head, int j, int len) {
     const uint32_t heads = __ballot_sync(0xffffffffu, head);
-    const uint32_t after = (heads | ~km) & ~le;
-    const int len = (after ? __ffs(after) - 1 : 32) - lane;  // rows in the piece headed here
     const int np = __popc(heads), pos = __popc(heads & lt);
     bool ok = true;
     // rounds of at most half the ring: a round ends when its last stage is free, and
@@ -282,6 +290,19 @@ __device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage
     }
     return true;
   };
+  // kept rows of channels [j0, j1), j1 - j0 <= 32, in pieces of up to rmax adjacent rows
+  auto issue = [&](int j0, int j1) {
+    const int j = j0 + lane;
+    const bool k = j < j1 && kept(j);
+    const uint32_t km = __ballot_sync(0xffffffffu, k);
+    const uint32_t runs = km & ~(km << 1);                 // first lanes of runs of kept channels
+    const int rs = 31 - __clz(runs & le);                  // start of this lane's run (if kept)
+    const bool head = k && ((lane - rs) % rmax == 0);      // first lane of a piece
+    const uint32_t heads = __ballot_sync(0xffffffffu, head);
+    const uint32_t after = (heads | ~km) & ~le;
+    const int len = (after ? __ffs(after) - 1 : 32) - lane;  // rows in the piece headed here
+    return issue_pieces(head, j, len);
+  };
   bool ok = true;
   const unsigned ndyn = wk.base < wk.n ? (unsigned)(wk.n - wk.base) : 0u;
   auto width = [&](unsigned taken) {
@@ -320,6 +341,15 @@ __device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage
         ok = false;
         break;
       }
+    }
+  }
+  if (ok && tail.ready) {
+    if (lane == 0) ok = mbar_wait(tail.ready, 0u);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    const int nt = ok ? *tail.n : 0;
+    for (int c0 = 0; c0 < nt && ok; c0 += 32) {
+      const bool v = c0 + lane < nt;
+      ok = issue_pieces(v, v ? tail.list[c0 + lane] : 0, 1);
     }
   }
   if (!__all_sync(0xffffffffu, ok)) return false;
@@ -385,17 +415,26 @@ __device__ bool consume_t(const Ring& R, int S, uint32_t row_bytes, uint32_t sta
       const int nr = R.meta_cnt[s];
       rows += nr;
       const uint32_t src = ring + (uint32_t)s * stage_bytes;
-      for (int r = 0; r < nr; ++r) {
-        const float xv = vals[row + r];
-        uint4 w[VPT];
+      // up to RU rows of the piece at a time: all their loads first, then the arithmetic
+      constexpr int RU = VPT <= 2 ? 4 : 1;
+      for (int r0 = 0; r0 < nr; r0 += RU) {
+        float xv[RU];
+        uint4 w[RU][VPT];
 #pragma unroll
-        for (int j = 0; j < VPT; ++j) {
-          const int v = t + j * kCT;
-          if (v < V) w[j] = ld_shared_u4(src + (uint32_t)r * row_bytes + (uint32_t)v * 16u);
+        for (int u = 0; u < RU; ++u) {
+          const int r = r0 + u;
+          xv[u] = r < nr ? vals[row + r] : 0.f;
+#pragma unroll
+          for (int j = 0; j < VPT; ++j) {
+            const int v = t + j * kCT;
+            if (r < nr && v < V) w[u][j] = ld_shared_u4(src + (uint32_t)r * row_bytes + (uint32_t)v * 16u);
+          }
         }
 #pragma unroll
-        for (int j = 0; j < VPT; ++j)
-          if (t + j * kCT < V) VecOps<BF16>::fma(acc[j], w[j], xv);
+        for (int u = 0; u < RU; ++u)
+#pragma unroll
+          for (int j = 0; j < VPT; ++j)
+            if (r0 + u < nr && t + j * kCT < V) VecOps<BF16>::fma(acc[j], w[u][j], xv[u]);
       }
     }
     __syncwarp();
@@ -423,14 +462,13 @@ __device__ bool consume(const Ring& R, int S, uint32_t row_bytes, uint32_t stage
                         const float* vals, float* out, unsigned long long* trace = nullptr) {
   constexpr int EPV = VecOps<BF16>::EPV;
   const int V = m / EPV;
+  // rows of at most kMaxVpt vectors per consumer thread (the host sends wider shapes to
+  // the batched path): the widest case sets the kernel's register budget
   switch ((V + kCT - 1) / kCT) {
     case 1: return consume_t<BF16, 1>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
     case 2: return consume_t<BF16, 2>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
     case 3: return consume_t<BF16, 3>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
-    case 4: return consume_t<BF16, 4>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
-    case 5: return consume_t<BF16, 5>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
-    case 6: return consume_t<BF16, 6>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
-    default: return consume_t<BF16, 8>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
+    default: return consume_t<BF16, kMaxVpt>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
   }
 }
 
@@ -455,11 +493,11 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   R.full = reinterpret_cast<uint64_t*>(smraw + SL.bars);
   R.empty = R.full + kMaxStages;
   R.base = reinterpret_cast<char*>(smraw + SL.ring);
-  uint64_t* aux = R.full + 2 * kMaxStages;  // input staging copies
+  uint64_t* aux = R.full + 2 * kMaxStages;  // input staging copies; aux + 1: down selection done
   unsigned char* stage_in = smraw + SL.stage;
   __shared__ uint32_t red[2 * kFT / 32 + 8];
   __shared__ double dred[3 * kFT / 32];
-  __shared__ int s_abort, s_last;
+  __shared__ int s_abort, s_last, s_ntail;
 
   const int G = gridDim.x, b = blockIdx.x;
   const int warp = threadIdx.x >> 5;
@@ -473,6 +511,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       mbar_init(&R.empty[s], (uint32_t)kCW);
     }
     mbar_init(aux, 1u);
+    mbar_init(aux + 1, 1u);  // the down selection is finished (overlapped phase E)
     mbar_init_fence();
     s_abort = 0;
   }
@@ -548,7 +587,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
     }
   }
   __syncthreads();
-  if (rank == (gate ? a.Gg : G - a.Gg) - 1) write_keep_bytes(flags, d, gate ? a.keep_g : a.keep_u);
+  if (rank == (gate ? a.Gg : G - a.Gg) - 1) write_keep_bytes(flags, d, gate ? a.keep_g : a.keep_u, kFT);
   stamp(a.stamps, 1);
   cta_time(a.cta_t, 0);
 
@@ -562,8 +601,9 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       const int cs = gate ? a.cs_g : a.cs_u, np = gate ? a.Gg : G - a.Gg;
       const PhaseWork wk{d, min(d, rank * cs), min(d, (rank + 1) * cs), min(d, np * cs), np, a.wmin_b,
                          a.ctr + (gate ? 0 : 1)};
+      auto kept = [&](int j) { return ((flags[j >> 5] >> (j & 31)) & 1u) != 0u; };
       const bool ok = produce(R, a.S_b, row_bytes, row_bytes, 1, reinterpret_cast<const char*>(gate ? a.wt_gate : a.wt_up),
-                              wk, flags, ps, pol, b == 0 ? a.trace : nullptr);
+                              wk, kept, ps, pol, b == 0 ? a.trace : nullptr);
       if (!ok && (threadIdx.x & 31) == 0) s_abort = 1;
     } else {
       if (!consume<BF16>(R, a.S_b, row_bytes, row_bytes, ffn, full_par, vals, gate ? acc_g : acc_u,
@@ -644,8 +684,21 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       }
     }
     stamp(a.stamps, 4);
-    if (topk) {
-      select_topk_flags_radix<kFT>(keys, ffn, a.k_down, hist, cand, red, flags, b == 0 ? a.stamps + 14 : nullptr);
+  }
+  // The down selection's boundary bin; with it known, rows surely kept (scores above
+  // the bin) can stream while the consumer warps finish the selection.
+  const bool topk = a.mode == WINA_GATE_TOPK;
+  const bool split = topk && a.k_down > 0 && a.k_down < ffn;
+  Crossing cr{0, 0u, 0u};
+  if (split) cr = radix_crossing<kFT>(hist, a.k_down, red);
+  stamp(a.stamps, 14);
+  const bool overlap = split && cr.cnt <= (uint32_t)kSelCand;
+  const uint32_t rb_e = (uint32_t)d * ESZ;
+  if (!overlap) {
+    if (split) {
+      select_general_flags<kFT>(keys, ffn, a.k_down, hist, cand, red, flags);
+    } else if (topk) {
+      select_topk_flags_radix<kFT>(keys, ffn, a.k_down, hist, cand, red, flags);
     } else {
       __syncthreads();
       if (a.mode == WINA_GATE_STAT)
@@ -653,17 +706,14 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       else
         flags_all(ffn, flags);
     }
-  }
-  __syncthreads();
-  stamp(a.stamps, 5);
-  if (b == G - 1) write_keep_bytes(flags, ffn, a.keep_d);
-  stamp(a.stamps, 6);
-  cta_time(a.cta_t, 2);
-
-  // ---------------- E: stream kept down rows through the ring ----------------
-  {
+    __syncthreads();
+    stamp(a.stamps, 5);
+    if (b == G - 1) write_keep_bytes(flags, ffn, a.keep_d, kFT);
+    stamp(a.stamps, 6);
+    cta_time(a.cta_t, 2);
+    // ---------------- E: stream kept down rows through the ring ----------------
     // the down scores are no longer needed: the ring now starts at keys
-    const uint32_t row_bytes = (uint32_t)d * ESZ, stage_bytes = (uint32_t)a.rows_e * row_bytes;
+    const uint32_t stage_bytes = (uint32_t)a.rows_e * rb_e;
     const int S = min(kMaxStages, (int)(((uint32_t)a.smem - SL.keys) / stage_bytes));
     Ring RE = R;
     RE.base = reinterpret_cast<char*>(smraw + SL.keys);
@@ -673,12 +723,56 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       const PhaseWork wk{ffn, min(ffn, b * a.cs_e), min(ffn, (b + 1) * a.cs_e), min(ffn, G * a.cs_e), G, a.wmin_e,
                          a.ctr + 2};
-      if (!produce(RE, S, row_bytes, stage_bytes, a.rows_e, reinterpret_cast<const char*>(a.wt_down), wk, flags, ps,
-                   pol) &&
+      auto kept = [&](int j) { return ((flags[j >> 5] >> (j & 31)) & 1u) != 0u; };
+      if (!produce(RE, S, rb_e, stage_bytes, a.rows_e, reinterpret_cast<const char*>(a.wt_down), wk, kept, ps, pol) &&
           (threadIdx.x & 31) == 0)
         s_abort = 1;
     } else {
-      if (!consume<BF16>(RE, S, row_bytes, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
+      if (!consume<BF16>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
+    }
+  } else {
+    // ---------------- D/E overlapped ----------------
+    // The ring lies past the selection's scratch (keys, hist and cand stay intact).
+    // Producer: rows whose score bin is above the boundary bin (kept whatever the
+    // selection's finish decides), as its own block and units; then, once the
+    // consumers have finished the selection, its share (channel mod G == b) of the kept
+    // boundary-bin rows. Consumers: finish the selection (named barrier over the 16
+    // consumer warps), list that share, then consume the ring.
+    const uint32_t stage_bytes = (uint32_t)a.rows_o * rb_e;
+    const uint32_t at = SL.stage;
+    const int S = min(kMaxStages, (int)(((uint32_t)a.smem - at) / stage_bytes));
+    Ring RE = R;
+    RE.base = reinterpret_cast<char*>(smraw + at);
+    int* tail = reinterpret_cast<int*>(cand);  // written once the finish no longer needs cand
+    uint64_t* sel_done = aux + 1;
+    if (producer) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const PhaseWork wk{ffn, min(ffn, b * a.cs_e), min(ffn, (b + 1) * a.cs_e), min(ffn, G * a.cs_e), G, a.wmin_e,
+                         a.ctr + 2};
+      const uint32_t B = (uint32_t)cr.bin;
+      auto sure = [&](int j) { return (keys[j] >> 19) > B; };
+      if (!produce(RE, S, rb_e, stage_bytes, a.rows_o, reinterpret_cast<const char*>(a.wt_down), wk, sure, ps, pol,
+                   nullptr, Tail{sel_done, tail, &s_ntail}) &&
+          (threadIdx.x & 31) == 0)
+        s_abort = 1;
+    } else {
+      radix_finish<kCT>(keys, ffn, a.k_down, cr, hist, cand, flags, ConsumerSync{},
+                        b == 0 ? a.stamps + 14 : nullptr);
+      // this CTA's share of the kept boundary-bin channels
+      if (threadIdx.x == 0) s_ntail = 0;
+      ConsumerSync{}();
+      const uint32_t* lst = hist;  // the bin's (key, channel) pairs, left by the finish
+      for (uint32_t e = threadIdx.x; e < cr.cnt; e += kCT) {
+        const uint32_t ch = lst[2 * e + 1];
+        if ((int)(ch % (uint32_t)G) == b && ((flags[ch >> 5] >> (ch & 31)) & 1u)) tail[atomicAdd(&s_ntail, 1)] = (int)ch;
+      }
+      ConsumerSync{}();
+      if (threadIdx.x == 0) mbar_arrive(sel_done);  // release: the list and its length
+      stamp(a.stamps, 5);
+      if (b == G - 1) write_keep_bytes(flags, ffn, a.keep_d, kCT);
+      stamp(a.stamps, 6);
+      cta_time(a.cta_t, 2);
+      if (!consume<BF16>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
     }
   }
   __syncthreads();
@@ -789,7 +883,12 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
     // at least two stages in the ring, which then starts at keys
     const uint32_t rb_e = (uint32_t)d * esz;
     const int rows_e = SLay.keys < kMaxSmem ? (int)std::min<size_t>(4, (kMaxSmem - SLay.keys) / (2 * (size_t)rb_e)) : 0;
-    if (G >= 2 && S_b >= 2 && rows_e >= 1) {
+    // overlapped with the down selection, the ring starts past the selection's scratch
+    const int rows_o = SLay.stage < kMaxSmem ? (int)std::min<size_t>(2, (kMaxSmem - SLay.stage) / (2 * (size_t)rb_e)) : 0;
+    // consumer threads hold at most kMaxVpt 16-byte vectors of a row (ffn and d elements)
+    const bool narrow = ((int64_t)ffn * esz / 16 + kCT - 1) / kCT <= kMaxVpt &&
+                        ((int64_t)d * esz / 16 + kCT - 1) / kCT <= kMaxVpt;
+    if (narrow && G >= 2 && S_b >= 2 && rows_e >= 1 && rows_o >= 1) {
       FfnParams p;
       p.wt_gate = f->wt_gate;
       p.wt_up = f->wt_up;
@@ -830,6 +929,7 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
       p.wmin_e = min_width(ffn, kept_e, 2.0);
       p.S_b = S_b;
       p.rows_e = rows_e;
+      p.rows_o = rows_o;
       p.smem = (int)smem;
       p.bar = reinterpret_cast<GridBarrier*>(w + L.bar);
       p.ctr = reinterpret_cast<unsigned*>(w + L.ctr);
