@@ -457,11 +457,12 @@ __device__ bool consume_t(const Ring& R, int S, uint32_t row_bytes, uint32_t sta
   return ok;
 }
 
-template <bool BF16>
+template <bool BF16, int VF>
 __device__ bool consume(const Ring& R, int S, uint32_t row_bytes, uint32_t stage_bytes, int m, uint32_t& full_par,
                         const float* vals, float* out, unsigned long long* trace = nullptr) {
   constexpr int EPV = VecOps<BF16>::EPV;
   const int V = m / EPV;
+  if constexpr (VF > 0) return consume_t<BF16, VF>(R, S, row_bytes, stage_bytes, V, full_par, vals, out, trace);
   // rows of at most kMaxVpt vectors per consumer thread (the host sends wider shapes to
   // the batched path): the widest case sets the kernel's register budget
   switch ((V + kCT - 1) / kCT) {
@@ -476,7 +477,12 @@ __device__ bool consume(const Ring& R, int S, uint32_t row_bytes, uint32_t stage
 // the kernel
 // ------------------------------------------------------------------------------------
 
-template <bool BF16>
+// MODE: the gate mode when fixed at compile time, or -1 (read from the parameters).
+// VB / VE: 16-byte vectors per consumer thread of a gate/up row and of a down row when
+// fixed, or 0 (dispatched at run time). The hot case (bf16, top-K, d <= 4096) gets its
+// own instantiations: only the code it runs, so fewer registers and a smaller
+// instruction footprint for the streaming loops.
+template <bool BF16, int MODE, int VB, int VE>
 __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   constexpr uint32_t ESZ = BF16 ? 2u : 4u;
   extern __shared__ __align__(128) unsigned char smraw[];
@@ -542,7 +548,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
     // x and this projection's c arrive by bulk copies (x into the staging buffer, c into
     // the keys buffer, where each score then replaces its c in place); meanwhile the
     // histogram is cleared. An x that is not 16-byte aligned is loaded by the threads.
-    const bool topk = a.mode == WINA_GATE_TOPK;
+    const bool topk = MODE >= 0 ? MODE == WINA_GATE_TOPK : a.mode == WINA_GATE_TOPK;
     const uint32_t xbytes = (uint32_t)d * (a.xdt == WINA_BF16 ? 2u : 4u);
     const bool xbulk = ((uintptr_t)a.x & 15u) == 0;
     if (threadIdx.x == 0) {
@@ -578,7 +584,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
     if (topk) {
       select_topk_flags_radix<kFT>(keys, d, gate ? a.k_gate : a.k_up, hist, cand, red, flags,
                                    b == 0 ? a.stamps + 12 : nullptr);
-    } else {
+    } else if constexpr (MODE != WINA_GATE_TOPK) {
       __syncthreads();
       if (a.mode == WINA_GATE_STAT)
         flags_from_threshold(vals, d, spark_threshold(vals, d, a.z, dred), flags);
@@ -606,8 +612,8 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
                               wk, kept, ps, pol, b == 0 ? a.trace : nullptr);
       if (!ok && (threadIdx.x & 31) == 0) s_abort = 1;
     } else {
-      if (!consume<BF16>(R, a.S_b, row_bytes, row_bytes, ffn, full_par, vals, gate ? acc_g : acc_u,
-                         b == 0 ? a.trace : nullptr))
+      if (!consume<BF16, VB>(R, a.S_b, row_bytes, row_bytes, ffn, full_par, vals, gate ? acc_g : acc_u,
+                             b == 0 ? a.trace : nullptr))
         s_abort = 1;
     }
   }
@@ -620,12 +626,12 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   stamp(a.stamps, 2);
   cta_time(a.cta_t, 1);
   // the ring is drained: fetch c_down into the staging buffer while waiting for the grid
-  if (threadIdx.x == 0 && a.mode == WINA_GATE_TOPK) {
+  if (threadIdx.x == 0 && (MODE >= 0 ? MODE == WINA_GATE_TOPK : a.mode == WINA_GATE_TOPK)) {
     mbar_expect_tx(aux, (uint32_t)ffn * 4u);
     bulk_copy_g2s(stage_in, a.c_down, (uint32_t)ffn * 4u, aux, pol);
   }
   if (!grid_sync_fixed(a.bar, G, a.status)) {
-    if (threadIdx.x == 0 && a.mode == WINA_GATE_TOPK) {  // let the issued copy land before exiting
+    if (threadIdx.x == 0 && (MODE >= 0 ? MODE == WINA_GATE_TOPK : a.mode == WINA_GATE_TOPK)) {  // let the issued copy land before exiting
       mbar_arrive(aux);
       mbar_wait(aux, 1u);
     }
@@ -642,7 +648,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   {
     // g into vals, u into keys (bulk copies); h replaces g and the score replaces u in
     // place; the score histogram is filled on the way
-    const bool topk = a.mode == WINA_GATE_TOPK;
+    const bool topk = MODE >= 0 ? MODE == WINA_GATE_TOPK : a.mode == WINA_GATE_TOPK;
     if (threadIdx.x == 0) {
       // the sums were made by other SMs' atomics (generic proxy); order them before the
       // bulk copies (async proxy) that read them
@@ -687,7 +693,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   }
   // The down selection's boundary bin; with it known, rows surely kept (scores above
   // the bin) can stream while the consumer warps finish the selection.
-  const bool topk = a.mode == WINA_GATE_TOPK;
+  const bool topk = MODE >= 0 ? MODE == WINA_GATE_TOPK : a.mode == WINA_GATE_TOPK;
   const bool split = topk && a.k_down > 0 && a.k_down < ffn;
   Crossing cr{0, 0u, 0u};
   if (split) cr = radix_crossing<kFT>(hist, a.k_down, red);
@@ -699,7 +705,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       select_general_flags<kFT>(keys, ffn, a.k_down, hist, cand, red, flags);
     } else if (topk) {
       select_topk_flags_radix<kFT>(keys, ffn, a.k_down, hist, cand, red, flags);
-    } else {
+    } else if constexpr (MODE != WINA_GATE_TOPK) {
       __syncthreads();
       if (a.mode == WINA_GATE_STAT)
         flags_from_threshold(vals, ffn, spark_threshold(vals, ffn, a.z, dred), flags);
@@ -728,7 +734,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
           (threadIdx.x & 31) == 0)
         s_abort = 1;
     } else {
-      if (!consume<BF16>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
+      if (!consume<BF16, VE>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
     }
   } else {
     // ---------------- D/E overlapped ----------------
@@ -772,7 +778,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       if (b == G - 1) write_keep_bytes(flags, ffn, a.keep_d, kCT);
       stamp(a.stamps, 6);
       cta_time(a.cta_t, 2);
-      if (!consume<BF16>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
+      if (!consume<BF16, VE>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
     }
   }
   __syncthreads();
@@ -877,8 +883,17 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
     const uint32_t rb_b = (uint32_t)ffn * esz;
     const int S_b = (int)std::min<size_t>(kMaxStages, ring / rb_b);
     const size_t smem = kMaxSmem;
-    const int G = bf16 ? max_coresident_grid(k_ffn_fused<true>, kFT, smem)
-                       : max_coresident_grid(k_ffn_fused<false>, kFT, smem);
+    // the specialised instantiation for bf16 top-K with one vector per thread of a down
+    // row, else the general one
+    const int vb = (int)(((int64_t)ffn * esz / 16 + kCT - 1) / kCT), ve = (int)(((int64_t)d * esz / 16 + kCT - 1) / kCT);
+    void (*kern)(FfnParams) = bf16 ? k_ffn_fused<true, -1, 0, 0> : k_ffn_fused<false, -1, 0, 0>;
+    if (bf16 && mode == WINA_GATE_TOPK && ve == 1) {
+      if (vb == 1) kern = k_ffn_fused<true, WINA_GATE_TOPK, 1, 1>;
+      else if (vb == 2) kern = k_ffn_fused<true, WINA_GATE_TOPK, 2, 1>;
+      else if (vb == 3) kern = k_ffn_fused<true, WINA_GATE_TOPK, 3, 1>;
+      else if (vb == 4) kern = k_ffn_fused<true, WINA_GATE_TOPK, 4, 1>;
+    }
+    const int G = max_coresident_grid(kern, kFT, smem);
     // phase E: rows per stage (pieces of up to that many adjacent rows per bulk copy),
     // at least two stages in the ring, which then starts at keys
     const uint32_t rb_e = (uint32_t)d * esz;
@@ -946,9 +961,7 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
       p.done = reinterpret_cast<unsigned*>(w + L.ctr) + 3;
       p.epoch = reinterpret_cast<unsigned*>(w + L.ctr) + 4;
       p.status = status_dev;
-      cudaError_t e = bf16 ? launch_kernel(k_ffn_fused<true>, dim3(G), dim3(kFT), smem, st, true, p)
-                           : launch_kernel(k_ffn_fused<false>, dim3(G), dim3(kFT), smem, st, true, p);
-      return cuda_status(e);
+      return cuda_status(launch_kernel(kern, dim3(G), dim3(kFT), smem, st, true, p));
     }
   }
 
