@@ -42,6 +42,7 @@ constexpr int kCT = kCW * 32;            // consumer threads
 constexpr int kFT = kCT + 32;            // threads per CTA (consumers + one producer warp)
 constexpr int kMaxStages = 16;           // ring stages at most
 constexpr int kMaxVpt = 4;               // 16-byte row vectors per consumer thread at most
+constexpr int kMaxPieces = 4;            // copy pieces (and rows) per ring stage at most
 constexpr size_t kMaxSmem = 224 * 1024;  // dynamic SMEM per CTA (227 KB per block on sm_100, less static)
 
 struct FfnParams {
@@ -65,6 +66,7 @@ struct FfnParams {
   int rows_o;            // the same when phase E overlaps the down selection (smaller ring)
   int smem;              // dynamic SMEM bytes of the launch
   int S_b;            // ring stages in phase B
+  int rows_b;         // phase B: rows per ring stage
   GridBarrier* bar;
   unsigned* ctr;  // [3] channel counters of the dynamic units: gate, up, down
   float* h;
@@ -83,7 +85,7 @@ struct FfnParams {
 };
 
 struct SmemLayout {
-  uint32_t vals, flags, meta_row, meta_cnt, bars, keys, ring, hist, cand, stage;
+  uint32_t vals, flags, meta_np, meta_row, meta_cnt, bars, keys, ring, hist, cand, stage;
 };
 
 // vals | flags | stage metadata | mbarriers | keys | ring. The selection's histogram and
@@ -104,8 +106,9 @@ __host__ __device__ inline SmemLayout ffn_smem_layout(int d, int ffn) {
   };
   L.vals = take(nb * 4, 16);
   L.flags = take((nb + 31) / 32 * 4, 16);
-  L.meta_row = take(kMaxStages * 4, 16);
-  L.meta_cnt = take(kMaxStages * 4, 16);
+  L.meta_np = take(kMaxStages * 4, 16);
+  L.meta_row = take(kMaxStages * kMaxPieces * 4, 16);
+  L.meta_cnt = take(kMaxStages * kMaxPieces * 4, 16);
   L.bars = take((2 * kMaxStages + 2) * 8, 16);
   L.keys = take(nb * 4, 128);
   L.ring = take(0, 128);
@@ -190,17 +193,19 @@ __device__ double spark_threshold(const float* v, int n, double z, double* dred)
 // ------------------------------------------------------------------------------------
 // the row ring: producer and consumers
 // ------------------------------------------------------------------------------------
-// Kept channels that follow one another have adjacent rows in the input-major layout.
-// A stage holds a piece of up to `rmax` such rows, fetched by one bulk copy: bulk copies
-// of short rows at scattered addresses stream well below HBM bandwidth, contiguous
-// copies of 16 KB and more reach it (so rmax > 1 for the short down rows).
+// Kept channels that follow one another have adjacent rows in the input-major layout;
+// a piece is a run of up to `rmax` such rows, fetched by one bulk copy (bulk copies of
+// short rows at scattered addresses stream well below HBM bandwidth, contiguous copies
+// of 16 KB and more reach it). A stage holds up to `rmax` rows in one or more pieces:
+// its consumers' fixed cost per stage (the barrier hand-offs) is paid once for them all.
 
 struct Ring {
-  char* base;      // SMEM
-  uint64_t* full;  // [kMaxStages]
+  char* base;       // SMEM
+  uint64_t* full;   // [kMaxStages]
   uint64_t* empty;  // [kMaxStages]
-  int* meta_row;    // first row of the piece in each stage, -1 = end of phase
-  int* meta_cnt;    // rows in the piece
+  int* meta_np;     // pieces in each stage, -1 = end of phase
+  int* meta_row;    // [kMaxStages][kMaxPieces] first row of each piece
+  int* meta_cnt;    // [kMaxStages][kMaxPieces] rows in each piece
 };
 
 // Producer state kept across phases (per-stage mbarrier parities).
@@ -242,52 +247,96 @@ __device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u, le = lt | (1u << lane);
   int stage = 0;
-  // this lane heads a piece of `len` rows starting at row j (if head); issue them all
+  // this lane heads a piece of `len` rows starting at row j (if head): pack the pieces,
+  // in lane order, into stages of at most rmax rows and issue them stage by stage
   auto issue_pieces = [&](bool head, int j, int len) {
     const uint32_t heads = __ballot_sync(0xffffffffu, head);
-    const int np = __popc(heads), pos = __popc(heads & lt);
-    bool ok = true;
-    // rounds of at most half the ring: a round ends when its last stage is free, and
-    // the other half of the ring stays in flight meanwhile
-    const int RS = max(1, S / 2);
-    for (int r0 = 0; r0 < np; r0 += RS) {
-      const int nr = min(RS, np - r0);
-      // each lane issues its piece as soon as its stage is free (the oldest first)
-      bool mine = head && pos >= r0 && pos < r0 + nr;
-      const int s = (stage + pos - r0) % S;
-      const bool was_used = (ps.used >> s) & 1u;
-      const uint32_t par = (ps.empty_par >> s) & 1u;
-      unsigned long long t0 = 0;
-      while (__any_sync(0xffffffffu, mine)) {
-        if (!mine) continue;
-        if (!was_used || mbar_test_wait(&R.empty[s], par)) {
-          const uint32_t bytes = (uint32_t)len * row_bytes;
-          R.meta_row[s] = j;
-          R.meta_cnt[s] = len;
-          mbar_arrive_expect_tx(&R.full[s], bytes);
-          bulk_copy_g2s(R.base + (size_t)s * stage_bytes, Wt + (size_t)j * row_bytes, bytes, &R.full[s], pol);
-          if (trace && stage + pos - r0 < 64) trace[stage + pos - r0] = globaltimer_ns();
-          mine = false;
-        } else {
-          const unsigned long long now = globaltimer_ns();
-          if (t0 == 0) {
-            t0 = now;
-          } else if (now - t0 > kPipeTimeoutNs) {
-            ok = false;
+    if (rmax == 1) {
+      // one row per stage: rounds of at most half the ring, each lane issuing its row as
+      // soon as its own stage is free (the oldest first); the other half of the ring
+      // stays in flight while a round waits
+      const int np = __popc(heads), pos = __popc(heads & lt);
+      const int RS = max(1, S / 2);
+      bool ok = true;
+      for (int r0 = 0; r0 < np; r0 += RS) {
+        const int nr = min(RS, np - r0);
+        bool mine = head && pos >= r0 && pos < r0 + nr;
+        const int s = (stage + pos - r0) % S;
+        const bool was_used = (ps.used >> s) & 1u;
+        const uint32_t par = (ps.empty_par >> s) & 1u;
+        unsigned long long t0 = 0;
+        while (__any_sync(0xffffffffu, mine)) {
+          if (!mine) continue;
+          if (!was_used || mbar_test_wait(&R.empty[s], par)) {
+            R.meta_row[s * kMaxPieces] = j;
+            R.meta_cnt[s * kMaxPieces] = 1;
+            R.meta_np[s] = 1;
+            mbar_arrive_expect_tx(&R.full[s], row_bytes);
+            bulk_copy_g2s(R.base + (size_t)s * stage_bytes, Wt + (size_t)j * row_bytes, row_bytes, &R.full[s], pol);
+            if (trace && stage + pos - r0 < 64) trace[stage + pos - r0] = globaltimer_ns();
             mine = false;
+          } else {
+            const unsigned long long now = globaltimer_ns();
+            if (t0 == 0) {
+              t0 = now;
+            } else if (now - t0 > kPipeTimeoutNs) {
+              ok = false;
+              mine = false;
+            }
           }
         }
+        for (int i = 0; i < nr; ++i) {  // the same state update in every lane
+          const int s2 = (stage + i) % S;
+          if ((ps.used >> s2) & 1u) ps.empty_par ^= 1u << s2;
+          ps.used |= 1u << s2;
+          ps.full_par ^= 1u << s2;
+        }
+        stage += nr;
+        if (__any_sync(0xffffffffu, !ok)) return false;
       }
-      // the same state update in every lane: nr consecutive stages were filled
-      for (int i = 0; i < nr; ++i) {
-        const int s = (stage + i) % S;
-        if ((ps.used >> s) & 1u) ps.empty_par ^= 1u << s;
-        ps.used |= 1u << s;
-        ps.full_par ^= 1u << s;
-      }
-      stage += nr;
-      if (__any_sync(0xffffffffu, !ok)) return false;
+      return true;
     }
+    int my_k = -1, my_off = 0, nst = 0, fill = rmax;
+    for (uint32_t hb = heads; hb; hb &= hb - 1u) {
+      const int l = __ffs(hb) - 1;
+      const int L = __shfl_sync(0xffffffffu, len, l);
+      if (fill + L > rmax) {
+        ++nst;
+        fill = 0;
+      }
+      if (lane == l) {
+        my_k = nst - 1;
+        my_off = fill;
+      }
+      fill += L;
+    }
+    for (int k = 0; k < nst; ++k) {
+      const int s = (stage + k) % S;
+      const bool mine = my_k == k;
+      const uint32_t pm = __ballot_sync(0xffffffffu, mine);
+      const uint32_t rows = __reduce_add_sync(0xffffffffu, mine ? (uint32_t)len : 0u);
+      bool ok = true;
+      if (lane == 0 && ((ps.used >> s) & 1u)) ok = mbar_wait_poll(&R.empty[s], (ps.empty_par >> s) & 1u);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+      if (mine) {
+        const int idx = __popc(pm & lt);
+        R.meta_row[s * kMaxPieces + idx] = j;
+        R.meta_cnt[s * kMaxPieces + idx] = len;
+      }
+      if (lane == 0) R.meta_np[s] = __popc(pm);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&R.full[s], rows * row_bytes);
+      __syncwarp();
+      if (mine) {
+        bulk_copy_g2s(R.base + (size_t)s * stage_bytes + (size_t)my_off * row_bytes, Wt + (size_t)j * row_bytes,
+                      (uint32_t)len * row_bytes, &R.full[s], pol);
+        if (trace && stage + k < 64) trace[stage + k] = globaltimer_ns();
+      }
+      if ((ps.used >> s) & 1u) ps.empty_par ^= 1u << s;
+      ps.used |= 1u << s;
+      ps.full_par ^= 1u << s;
+    }
+    stage += nst;
     return true;
   };
   // kept rows of channels [j0, j1), j1 - j0 <= 32, in pieces of up to rmax adjacent rows
@@ -358,8 +407,7 @@ __device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage
     const int s = stage % S;
     if ((ps.used >> s) & 1u) ok = mbar_wait(&R.empty[s], (ps.empty_par >> s) & 1u);
     if (ok) {
-      R.meta_row[s] = -1;
-      R.meta_cnt[s] = 0;
+      R.meta_np[s] = -1;
       mbar_arrive(&R.full[s]);
     }
   }
@@ -410,11 +458,11 @@ __device__ bool consume_t(const Ring& R, int S, uint32_t row_bytes, uint32_t sta
     }
     if (trace && t == 0 && stage < 64) trace[64 + stage] = globaltimer_ns();
     full_par ^= 1u << s;
-    const int row = R.meta_row[s];
-    if (row >= 0) {
-      const int nr = R.meta_cnt[s];
+    const int np = R.meta_np[s];
+    uint32_t src = ring + (uint32_t)s * stage_bytes;
+    for (int p = 0; p < np; ++p) {
+      const int row = R.meta_row[s * kMaxPieces + p], nr = R.meta_cnt[s * kMaxPieces + p];
       rows += nr;
-      const uint32_t src = ring + (uint32_t)s * stage_bytes;
       // up to RU rows of the piece at a time: all their loads first, then the arithmetic
       constexpr int RU = VPT <= 2 ? 4 : 1;
       for (int r0 = 0; r0 < nr; r0 += RU) {
@@ -436,10 +484,11 @@ __device__ bool consume_t(const Ring& R, int S, uint32_t row_bytes, uint32_t sta
           for (int j = 0; j < VPT; ++j)
             if (r0 + u < nr && t + j * kCT < V) VecOps<BF16>::fma(acc[j], w[u][j], xv[u]);
       }
+      src += (uint32_t)nr * row_bytes;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&R.empty[s]);
-    if (row < 0) break;
+    if (np < 0) break;
     ++stage;
   }
   if (rows == 0) return ok;  // nothing to add
@@ -494,6 +543,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   uint32_t* hist = reinterpret_cast<uint32_t*>(smraw + SL.hist);
   uint32_t* cand = reinterpret_cast<uint32_t*>(smraw + SL.cand);
   Ring R;
+  R.meta_np = reinterpret_cast<int*>(smraw + SL.meta_np);
   R.meta_row = reinterpret_cast<int*>(smraw + SL.meta_row);
   R.meta_cnt = reinterpret_cast<int*>(smraw + SL.meta_cnt);
   R.full = reinterpret_cast<uint64_t*>(smraw + SL.bars);
@@ -608,11 +658,12 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       const PhaseWork wk{d, min(d, rank * cs), min(d, (rank + 1) * cs), min(d, np * cs), np, a.wmin_b,
                          a.ctr + (gate ? 0 : 1)};
       auto kept = [&](int j) { return ((flags[j >> 5] >> (j & 31)) & 1u) != 0u; };
-      const bool ok = produce(R, a.S_b, row_bytes, row_bytes, 1, reinterpret_cast<const char*>(gate ? a.wt_gate : a.wt_up),
+      const bool ok = produce(R, a.S_b, row_bytes, (uint32_t)a.rows_b * row_bytes, a.rows_b,
+                              reinterpret_cast<const char*>(gate ? a.wt_gate : a.wt_up),
                               wk, kept, ps, pol, b == 0 ? a.trace : nullptr);
       if (!ok && (threadIdx.x & 31) == 0) s_abort = 1;
     } else {
-      if (!consume<BF16, VB>(R, a.S_b, row_bytes, row_bytes, ffn, full_par, vals, gate ? acc_g : acc_u,
+      if (!consume<BF16, VB>(R, a.S_b, row_bytes, (uint32_t)a.rows_b * row_bytes, ffn, full_par, vals, gate ? acc_g : acc_u,
                              b == 0 ? a.trace : nullptr))
         s_abort = 1;
     }
@@ -881,7 +932,10 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
     size_t ring = SLay.ring < kMaxSmem ? (kMaxSmem - SLay.ring) / 128 * 128 : 0;
     if (ring < ffn_min_ring((int)d, (int)ffn)) ring = 0;
     const uint32_t rb_b = (uint32_t)ffn * esz;
-    const int S_b = (int)std::min<size_t>(kMaxStages, ring / rb_b);
+    // phase B: one row per stage (rows of ffn elements are long enough; more stages keep
+    // more bytes in flight while the ring refills)
+    const int rows_b = 1;
+    const int S_b = (int)std::min<size_t>(kMaxStages, ring / ((size_t)rows_b * rb_b));
     const size_t smem = kMaxSmem;
     // the specialised instantiation for bf16 top-K with one vector per thread of a down
     // row, else the general one
@@ -899,7 +953,7 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
     const uint32_t rb_e = (uint32_t)d * esz;
     const int rows_e = SLay.keys < kMaxSmem ? (int)std::min<size_t>(4, (kMaxSmem - SLay.keys) / (2 * (size_t)rb_e)) : 0;
     // overlapped with the down selection, the ring starts past the selection's scratch
-    const int rows_o = SLay.stage < kMaxSmem ? (int)std::min<size_t>(2, (kMaxSmem - SLay.stage) / (2 * (size_t)rb_e)) : 0;
+    const int rows_o = SLay.stage < kMaxSmem ? (int)std::min<size_t>(4, (kMaxSmem - SLay.stage) / (2 * (size_t)rb_e)) : 0;
     // consumer threads hold at most kMaxVpt 16-byte vectors of a row (ffn and d elements)
     const bool narrow = ((int64_t)ffn * esz / 16 + kCT - 1) / kCT <= kMaxVpt &&
                         ((int64_t)d * esz / 16 + kCT - 1) / kCT <= kMaxVpt;
@@ -943,6 +997,7 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
       p.wmin_b = min_width(d, kept_b, 1.0);
       p.wmin_e = min_width(ffn, kept_e, 2.0);
       p.S_b = S_b;
+      p.rows_b = rows_b;
       p.rows_e = rows_e;
       p.rows_o = rows_o;
       p.smem = (int)smem;

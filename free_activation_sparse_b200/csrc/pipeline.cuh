@@ -76,6 +76,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// As mbar_wait, but polling without suspending the thread (for a producer that must
+// react as soon as a stage frees); false after the time limit.
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_test_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kPipeTimeoutNs) return false;
+  }
+  return true;
+}
+
 // Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
 // to this CTA's shared memory, completing `bytes` of transaction count on `bar`.
 __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,
