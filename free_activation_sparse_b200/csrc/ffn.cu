@@ -18,11 +18,8 @@
 //   C  Every CTA reads the complete g and u, computes h = silu(g) * u and the down
 //      gate's scores |h_j * c_down_j| for all ffn channels, and selects the kept down
 //      channels itself (bitmask).
-//   E  Every CTA takes an equal share of the kept down rows (by rank in index order)
-//      and streams them with 16-byte loads, 16 rows in flight per thread (rows of d
-//      elements are too short for bulk copies to reach HBM bandwidth); row sums are
-//      added into y's accumulator.
-//   F  The last CTA to finish (a counter) copies y out and clears the accumulators.
+//   E  As B over the down rows (d wide), several rows per stage; row sums are added
+//      straight into y (cleared by the CTAs before the grid barrier).
 // Every wait (grid barrier, ring stage) is bounded in time; on a timeout the kernel
 // records WINA_ERR_TIMEOUT, waits (bounded) for its own copies in flight and returns.
 // Several tokens: the batched calls (select, sparse_matvec, silu*mul, select,
@@ -78,8 +75,6 @@ struct FfnParams {
   unsigned long long* trace;  // CTA 0: phase B [0..63] issued, [64..127] ready; phase E [128..255]
   float* acc_g;     // [2][ffn] float32 sums of the gate rows, one buffer per call parity
   float* acc_u;     // [2][ffn] float32 sums of the up rows, one buffer per call parity
-  float* acc_y;     // [d] float32 sums of the down rows (zero between calls)
-  unsigned* done;   // CTAs that finished phase E (zero between calls)
   unsigned* epoch;  // calls completed on this workspace (picks the parity)
   int32_t* status;
 };
@@ -553,7 +548,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   unsigned char* stage_in = smraw + SL.stage;
   __shared__ uint32_t red[2 * kFT / 32 + 8];
   __shared__ double dred[3 * kFT / 32];
-  __shared__ int s_abort, s_last, s_ntail;
+  __shared__ int s_abort, s_ntail;
 
   const int G = gridDim.x, b = blockIdx.x;
   const int warp = threadIdx.x >> 5;
@@ -588,6 +583,10 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       __stcg(cg + q, make_float4(0.f, 0.f, 0.f, 0.f));
       __stcg(cu + q, make_float4(0.f, 0.f, 0.f, 0.f));
     }
+    // y receives the down rows' sums by atomics after the grid barrier: clear it now
+    for (int q = d * b / G + threadIdx.x; q < d * (b + 1) / G; q += kFT) __stcg(a.y + q, 0.f);
+    // the previous call has completed: its down-unit counter can start again
+    if (b == 0 && threadIdx.x == 0) a.ctr[2] = 0u;
   }
 
   // ---------------- A: this CTA's projection, its kept-channel bitmask ----------------
@@ -695,6 +694,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   if (b == 0 && threadIdx.x == 0) {
     a.ctr[0] = 0u;  // every CTA is past phase B: the gate/up unit counters can be reset
     a.ctr[1] = 0u;
+    *a.epoch = *a.epoch + 1u;  // every CTA has read it: the next call uses the other g/u buffers
   }
   {
     // g into vals, u into keys (bulk copies); h replaces g and the score replaces u in
@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
           (threadIdx.x & 31) == 0)
         s_abort = 1;
     } else {
-      if (!consume<BF16, VE>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
+      if (!consume<BF16, VE>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.y)) s_abort = 1;
     }
   } else {
     // ---------------- D/E overlapped ----------------
@@ -829,7 +829,7 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
       if (b == G - 1) write_keep_bytes(flags, ffn, a.keep_d, kCT);
       stamp(a.stamps, 6);
       cta_time(a.cta_t, 2);
-      if (!consume<BF16, VE>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.acc_y)) s_abort = 1;
+      if (!consume<BF16, VE>(RE, S, rb_e, stage_bytes, d, full_par, vals, a.y)) s_abort = 1;
     }
   }
   __syncthreads();
@@ -841,26 +841,6 @@ __global__ void __launch_bounds__(kFT, 1) k_ffn_fused(FfnParams a) {
   stamp(a.stamps, 7);
   cta_time(a.cta_t, 3);
 
-  // ---------------- F: the last CTA to finish writes y and clears the sums ----------------
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned old = atomicAdd(a.done, 1u);
-    s_last = old == (unsigned)(G - 1);
-    __threadfence();
-  }
-  __syncthreads();
-  if (s_last) {
-    for (int q = threadIdx.x; q < d / 4; q += kFT) {
-      float4* p = reinterpret_cast<float4*>(a.acc_y) + q;
-      reinterpret_cast<float4*>(a.y)[q] = __ldcg(p);
-      __stcg(p, make_float4(0.f, 0.f, 0.f, 0.f));
-    }
-    if (threadIdx.x == 0) {
-      a.ctr[2] = 0u;
-      *a.done = 0u;
-      *a.epoch = *a.epoch + 1u;  // the next call uses the other g/u buffers
-    }
-  }
   stamp(a.stamps, 8);
   stamp(a.stamps, 9);
 }
@@ -1012,8 +992,6 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
       p.trace = reinterpret_cast<unsigned long long*>(w + L.stamps) + 16;
       p.acc_g = reinterpret_cast<float*>(w + L.acc_g);
       p.acc_u = reinterpret_cast<float*>(w + L.acc_u);
-      p.acc_y = reinterpret_cast<float*>(w + L.acc_y);
-      p.done = reinterpret_cast<unsigned*>(w + L.ctr) + 3;
       p.epoch = reinterpret_cast<unsigned*>(w + L.ctr) + 4;
       p.status = status_dev;
       return cuda_status(launch_kernel(kern, dim3(G), dim3(kFT), smem, st, true, p));

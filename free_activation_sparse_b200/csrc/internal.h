@@ -89,15 +89,15 @@ inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
 }
 
 // sparse_ffn_swiglu (d, ffn, batch):
-//   bar | ctr [8] (unit counters, done, epoch) | h [B][ffn] | keep_g [B][d] | keep_u [B][d] (bytes)
+//   bar | ctr [8] (three unit counters, -, epoch) | h [B][ffn] | keep_g [B][d] | keep_u [B][d] (bytes)
 //   | keep_d [B][ffn] (bytes) | stamps [kFfnStamps] | cta_t [kGridCap][4]
 //   | idx_gate, idx_up [B][d] | idx_down [B][ffn] | cnt [3][B] | xs_gate, xs_up [B][d]
 //   | xs_down [B][ffn] | g, u [B][ffn]                       (several tokens)
-//   | acc_g, acc_u [2][ffn] | acc_y [d]                       (one token)
+//   | acc_g, acc_u [2][ffn]                                 (one token)
 //   | spmv ws                                                 (several tokens)
 struct FfnWs {
   size_t bar, ctr, h, keep_g, keep_u, keep_d, stamps, cta_t, idx_gate, idx_up, idx_down, cnt, xs_gate,
-      xs_up, xs_down, g, u, acc_g, acc_u, acc_y, spmv, total;
+      xs_up, xs_down, g, u, acc_g, acc_u, spmv, total;
 };
 inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   FfnWs w;
@@ -127,7 +127,6 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   w.u = take(one ? 0 : (size_t)B * ffn * 4);
   w.acc_g = take(one ? (size_t)2 * ffn * 4 : 0);
   w.acc_u = take(one ? (size_t)2 * ffn * 4 : 0);
-  w.acc_y = take(one ? (size_t)d * 4 : 0);
   const int64_t mmax = ffn > d ? ffn : d;
   w.spmv = take(one ? 0 : spmv_ws_layout(mmax, B).total);
   w.total = o;
