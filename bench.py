@@ -319,6 +319,47 @@ def main():
     us_layer_dense = dense_ms / nd * 1e3 / L
     del dgraph
 
+    # several tokens (the batched path): 16 tokens per call on the same layers; effective
+    # bytes count the union of each projection's kept rows over the tokens
+    BT = 16
+    xbs, yb = [], torch.empty((BT, D), dtype=torch.float32, device="cuda")
+    for l in range(L):
+        cfgb = synth.make_llama7b_ffn(batch=BT, p=args.p, layer=l + 1000 * rank)
+        xbs.append(torch.from_numpy(cfgb["x"].view(np.int16)).cuda().view(torch.bfloat16))
+    wsb = W.Workspace(W.OP_FFN_SWIGLU, D, FFN, 0, BT)
+
+    def batched_step():
+        for l in range(L):
+            W.sparse_ffn_swiglu(layers[l], xbs[l], W.GATE_TOPK, kg, kg, kd, ws=wsb, status=status, y=yb)
+
+    for _ in range(3):
+        batched_step()
+    union_bytes = 0
+    for l in range(L):  # the kept sets of every layer (read back from the call's own views)
+        W.sparse_ffn_swiglu(layers[l], xbs[l], W.GATE_TOPK, kg, kg, kd, ws=wsb, status=status, y=yb)
+        v = W.ffn_ws_view(wsb, D, FFN, BT)
+        ug, uu, ud = (int(v[k].bool().any(0).sum().item()) for k in ("keep_gate", "keep_up", "keep_down"))
+        union_bytes += (ug + uu) * FFN * 2 + ud * D * 2 + BT * (D * 2 + D * 4) + (2 * D + FFN) * 4
+    nb_steps = max(3, args.steps // 2)
+    barrier()
+    torch.cuda.synchronize()
+    t_b0 = torch.cuda.Event(enable_timing=True)
+    t_b1 = torch.cuda.Event(enable_timing=True)
+    t_b0.record(stream)
+    for _ in range(nb_steps):
+        batched_step()
+    t_b1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    batched_ms = max_over_ranks(t_b0.elapsed_time(t_b1))
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the batched run")
+    batched = {"batch": BT, "us_per_layer": batched_ms / nb_steps * 1e3 / L,
+               "effective_gbs": world * union_bytes * nb_steps / (batched_ms * 1e-3) / 1e9,
+               "union_bytes_per_layer": union_bytes // L,
+               "path": "batched calls (select, sparse product, silu*mul) per token group, eager"}
+    del xbs, yb, wsb
+
     # end to end through the C ABI: host x in pinned memory -> device, the call, y -> host
     hx = [x.cpu().pin_memory() for x in xs]
     hy = [torch.empty((1, D), dtype=torch.float32).pin_memory() for _ in range(L)]
@@ -368,6 +409,7 @@ def main():
         "eager": {"us_per_layer": eager_ms / max(3, args.steps // 2) * 1e3 / L,
                   "kernel_us_events": eager_kern_ms * 1e3},
         "dense": {"us_per_layer": us_layer_dense, "speedup": us_layer_dense / us_layer},
+        "batched": batched,
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "us_per_layer": e2e_ms / args.steps * 1e3 / L,
                 "h2d_bytes_per_step": L * D * 2, "d2h_bytes_per_step": L * D * 4},
         "gpu_launches": L * args.steps,

@@ -16,10 +16,13 @@
 //      float atomics at L2).
 //   -- grid barrier --
 //   C  Every CTA reads the complete g and u, computes h = silu(g) * u and the down
-//      gate's scores |h_j * c_down_j| for all ffn channels, and selects the kept down
-//      channels itself (bitmask).
-//   E  As B over the down rows (d wide), several rows per stage; row sums are added
-//      straight into y (cleared by the CTAs before the grid barrier).
+//      gate's scores |h_j * c_down_j| for all ffn channels, and finds the down
+//      selection's boundary score bin.
+//   D/E The producer warp starts streaming the down rows whose scores lie above that bin
+//      (kept whatever the rest of the selection decides) while the consumer warps finish
+//      the selection; then the CTA's share of the kept boundary-bin rows follows. Down
+//      rows are short, so a stage holds up to four of them in contiguous pieces. Row
+//      sums are added straight into y (cleared by the CTAs before the grid barrier).
 // Every wait (grid barrier, ring stage) is bounded in time; on a timeout the kernel
 // records WINA_ERR_TIMEOUT, waits (bounded) for its own copies in flight and returns.
 // Several tokens: the batched calls (select, sparse_matvec, silu*mul, select,
@@ -59,11 +62,11 @@ struct FfnParams {
   int Gg;             // CTAs on the gate projection in phase B
   int cs_g, cs_u, cs_e;  // channels in each CTA's own block: gate, up (phase B), down (E)
   int wmin_b, wmin_e;    // shortest dynamic unit (channels) in phases B and E
-  int rows_e;            // phase E: rows per ring stage (longest contiguous copy)
+  int rows_e;            // phase E: rows per ring stage (ring over keys and past them)
   int rows_o;            // the same when phase E overlaps the down selection (smaller ring)
   int smem;              // dynamic SMEM bytes of the launch
-  int S_b;            // ring stages in phase B
-  int rows_b;         // phase B: rows per ring stage
+  int S_b;               // ring stages in phase B
+  int rows_b;            // phase B: rows per ring stage
   GridBarrier* bar;
   unsigned* ctr;  // [3] channel counters of the dynamic units: gate, up, down
   float* h;
@@ -72,7 +75,7 @@ struct FfnParams {
   uint8_t* keep_d;
   long long* stamps;
   unsigned long long* cta_t;
-  unsigned long long* trace;  // CTA 0: phase B [0..63] issued, [64..127] ready; phase E [128..255]
+  unsigned long long* trace;  // CTA 0, phase B: [0..63] stage issued, [64..127] stage taken (ns)
   float* acc_g;     // [2][ffn] float32 sums of the gate rows, one buffer per call parity
   float* acc_u;     // [2][ffn] float32 sums of the up rows, one buffer per call parity
   unsigned* epoch;  // calls completed on this workspace (picks the parity)
@@ -84,9 +87,9 @@ struct SmemLayout {
 };
 
 // vals | flags | stage metadata | mbarriers | keys | ring. The selection's histogram and
-// candidate list, and the input staging buffer, overlay the start of the ring, which is
-// idle while a selection runs; in phase E the ring extends down over keys (past the
-// CTA's row list kept at its start).
+// candidate lists, and the input staging buffer, overlay the start of the ring, which is
+// idle while a selection runs. Phase E's ring starts past that scratch while it overlaps
+// the down selection, or at keys when it runs after a complete selection.
 __host__ __device__ inline SmemLayout ffn_smem_layout(int d, int ffn) {
   SmemLayout L;
   // room for max(d, ffn) channels, rounded up to 128 (the selection reads whole
@@ -220,20 +223,23 @@ struct PhaseWork {
   unsigned* ctr;
 };
 
-// Streams the phase's kept rows into the ring in pieces (see above), then an end-of-
-// phase marker. Runs on the producer warp. The pieces of a 32-channel window are issued
-// by as many lanes at once (a single thread issuing bulk copies one after another is
-// far too slow to fill HBM), in rounds of at most S so that the stages of a round are
-// distinct. The next unit is requested when a unit starts, so the counter's round trip
-// overlaps the unit's copies, and none is requested while the CTA's own block is
-// streamed. Returns false on a timeout.
-// The producer's tail: after its own block and units, the rows listed in tail[0..*tail_n)
-// (one row each), once `tail_ready` (an mbarrier) has completed its first phase.
+// The producer's tail: after its own block and units, the rows listed in list[0..*n)
+// (one row each), once `ready` (an mbarrier) has completed its first phase.
 struct Tail {
   uint64_t* ready;
   const int* list;
   const int* n;
 };
+
+// Streams the phase's kept rows (kept(j) true) into the ring in pieces (see above), then
+// an end-of-phase marker. Runs on the producer warp. The pieces of a 32-channel window
+// are issued by several lanes at once (a single thread issuing bulk copies one after
+// another is far too slow to fill HBM): with one row per stage, each lane issues its
+// row as soon as its own stage frees, in rounds of at most half the ring; with several
+// rows per stage, the window's pieces are packed into stages, each stage's copies
+// issued together once it frees. The first unit is requested halfway through the CTA's
+// own block and each next one when a unit starts, so the counter's round trip overlaps
+// the copies and no unit is held long. Returns false on a timeout.
 
 template <typename Kept>
 __device__ bool produce(const Ring& R, int S, uint32_t row_bytes, uint32_t stage_bytes, int rmax,

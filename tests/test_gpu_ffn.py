@@ -188,3 +188,27 @@ def test_gemma_stat_gate(gemma, B):
         assert rel_l2(y[b], O.sparse_matvec(Wdf, idn, h_gpu[idn].astype(np.float64))) <= TOL_STAGE
         e2e = O.ffn_swiglu(Wgf, Wuf, Wdf, None, None, None, x32[b], 0, 0, 0, mode="stat", s=s)
         assert rel_l2(y[b], e2e["y"]) <= TOL_E2E
+
+
+def test_all_scores_equal_take_the_general_search_and_lowest_indices():
+    # Constant weights and input: every gate/up score is equal, so is every h and every
+    # down score. The boundary bin then holds all keys (more than the exact-ranking
+    # room), the general search decides both selections, and ties keep the lowest
+    # channel indices.
+    d, ffn = 1024, 2048
+    one32 = np.full((ffn, d), 1.0 / 32.0, dtype=np.float32)
+    Wg = synth.bf16_bits_from_f32(one32)
+    Wu = synth.bf16_bits_from_f32(one32)
+    Wd = synth.bf16_bits_from_f32(np.full((d, ffn), 1.0 / 32.0, dtype=np.float32))
+    f = _prep_bf16(Wg, Wu, Wd)
+    Wgf, Wuf, Wdf = (O.widen_bf16(a) for a in (Wg, Wu, Wd))
+    x = np.ones((1, d), dtype=np.float32)
+    kg, ku, kd = 300, 700, 900
+    y = _check_topk_ffn(f, Wgf, Wuf, Wdf, dev_f32(x), x, kg, ku, kd)
+    ws = W.Workspace(W.OP_FFN_SWIGLU, d, ffn, 0, 1)
+    W.sparse_ffn_swiglu(f, dev_f32(x), W.GATE_TOPK, kg, ku, kd, ws=ws, y=dev_f32(np.zeros((1, d), np.float32)))
+    v = {k: host(t) for k, t in W.ffn_ws_view(ws, d, ffn, 1).items()}
+    assert np.array_equal(np.nonzero(v["keep_gate"][0])[0], np.arange(kg))
+    assert np.array_equal(np.nonzero(v["keep_up"][0])[0], np.arange(ku))
+    assert np.array_equal(np.nonzero(v["keep_down"][0])[0], np.arange(kd))
+    assert np.isfinite(y).all()
