@@ -248,11 +248,15 @@ wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt, int64_t n,
  *   S_d = gate(h, c_down, k_down);  y = W_down[:, S_d] h[S_d]
  * With WINA_GATE_STAT every gate is the Spark threshold with keep fraction s on the
  * projection's signed input (k_* ignored); with WINA_GATE_DENSE every channel is kept.
- * One token runs as one persistent cooperative kernel: each SM works on the gate or the
- * up projection, selects that projection's kept channels itself, takes small units of
- * channels from a global counter and streams their kept weight rows HBM -> SMEM with
- * bulk copies through a ring of stages; grid barriers (bounded waits) separate the
- * phases. Several tokens run as a sequence of the batched calls above.
+ * One token (with d, ffn at most 16384 bf16 / 8192 f32 elements) runs as one persistent
+ * cooperative kernel: each SM works on the gate or the up projection, selects that
+ * projection's kept channels itself, streams its own block of channels' kept weight rows
+ * HBM -> SMEM with bulk copies through a ring of stages, then takes units of channels from
+ * a global counter; one grid barrier (bounded wait) makes g and u complete; every SM then
+ * selects the down projection's kept channels itself and streams its share of those rows,
+ * adding into y. Kept sets are exact; y's float32 summation order is not fixed, so repeated
+ * calls agree to float32 rounding. Several tokens (or wider shapes) run as a sequence of
+ * the batched calls above.
  *   f:   host pointer to the weight descriptor (read during the call only).
  *   x:   device [batch][d] of xdt.   y: device float32 [batch][d] (written).
  *   k_gate, k_up in [0, d]; k_down in [0, ffn] (WINA_GATE_TOPK).  0 < s < 1 (STAT).
