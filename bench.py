@@ -8,9 +8,11 @@ so every step streams its kept rows from HBM.
 
 Printed (rank 0, one JSON line): effective HBM GB/s on the bytes the kept rows and the
 vectors require (value; whole job), us per layer, the roofline of the fused kernel
-against the measured HBM copy bandwidth, the dense comparator (the same kernel with
-every channel kept), the end-to-end figure through the C ABI with host buffers, and
-the CPU oracle's time on a bounded sample.
+against the measured HBM copy bandwidth (with the ncu DRAM traffic of one launch when
+profiles/ holds it for this kernel source), the dense comparator (the same kernel with
+every channel kept), 16 tokens per call on the batched path (against the union of the
+kept rows), the end-to-end figure through the C ABI with host buffers, and the CPU
+oracle's time on a bounded sample.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--p 0.5] [--layers 8]
   python bench.py --impl reference ...   # the CPU oracle, timed on the host cores
