@@ -18,7 +18,7 @@ Sources (web pages on training-free activation sparsity; cited by title and sect
   section "WAS框架的核心创新" (weight-aware sparsity applied per component:
   Q, K, V, O, gate, up, down).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * ties in the top-K gate go to the lower channel index; the kept set is returned as an
   ascending index list;
