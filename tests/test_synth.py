@@ -39,3 +39,18 @@ def test_weight_recipe_column_scale():
     col_std = w.std(axis=0)
     assert col_std.max() / col_std.min() > 1.2
     assert w.dtype == np.float32
+
+
+def test_bench_bytes_per_layer():
+    # The bench's unit: the kept rows of the three bf16 weights (Llama-7B FFN, d 4096,
+    # ffn 11008) plus the vectors that cross HBM (x bf16, c_gate/c_up/c_down and y float32).
+    import bench
+
+    rows_p50 = (2048 + 2048) * 11008 * 2 + 5504 * 4096 * 2
+    rows_p65 = (1434 + 1434) * 11008 * 2 + 3853 * 4096 * 2
+    assert rows_p50 == 135_266_304 and rows_p65 == 94_705_664
+    vecs = 4096 * 2 + 2 * 4096 * 4 + 11008 * 4 + 4096 * 4
+    assert bench.layer_bytes(2048, 2048, 5504) == rows_p50 + vecs == 135_367_680
+    kg, kd = synth.keep_count(0.65, 4096), synth.keep_count(0.65, 11008)
+    assert (kg, kd) == (1434, 3853)
+    assert bench.layer_bytes(kg, kg, kd) == rows_p65 + vecs
