@@ -45,6 +45,7 @@ __all__ = [
     "select_topk",
     "wina_select",
     "teal_select",
+    "svd_transform",
     "sparse_matvec",
     "sparse_matvec_rows",
     "dense_matvec",
@@ -250,6 +251,17 @@ def overlap(S, T) -> dict:
 # --------------------------------------------------------------------------------------
 # the approximation error the theorem speaks of ([WINA] section 二)
 # --------------------------------------------------------------------------------------
+
+
+def svd_transform(W):
+    """The column-orthogonalising transform of [WINA] section 五: with the thin SVD
+    W = U diag(s) V^T, W' = W V = U diag(s) has orthogonal columns (W'^T W' = diag(s^2),
+    column norms s), and W' (V^T x) = W x, so the gate can run on W' and x' = V^T x without
+    changing the layer's output. Returns (W', V) in float64. Offline; not on the path."""
+    W64 = np.asarray(W, dtype=np.float64)
+    _, _, vt = np.linalg.svd(W64, full_matrices=False)
+    V = vt.T
+    return W64 @ V, V
 
 
 def output_error(W, x, idx) -> float:

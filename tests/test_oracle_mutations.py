@@ -81,6 +81,13 @@ def _silu_minus(g):
         return g / (1.0 + np.exp(g))
 
 
+def _svd_transposed(Wm):
+    # transposed operand: W V^T instead of W V
+    W64 = np.asarray(Wm, dtype=np.float64)
+    _, _, vt = np.linalg.svd(W64, full_matrices=False)
+    return W64 @ vt, vt.T
+
+
 MUTATIONS = {
     "col_norms:row-norms": ("col_norms", _row_norms),
     "gate_scores:no-abs": ("gate_scores", _scores_no_abs),
@@ -91,6 +98,7 @@ MUTATIONS = {
     "spark:non-strict": ("spark_threshold", _spark_ge),
     "spark:wrong-tail": ("spark_threshold", _spark_wrong_tail),
     "silu:sign": ("silu", _silu_minus),
+    "svd_transform:transposed-V": ("svd_transform", _svd_transposed),
 }
 
 PINS = [
@@ -104,6 +112,8 @@ PINS = [
     P.test_ffn_identity_weights_hand_computed,
     P.test_gate_scores_single_fp32_multiply,
     lambda: P.test_spark_keep_fraction_gaussian(2304, 2e-3, 0.03),
+    P.test_svd_transform_orthogonal_columns_and_norms,
+    P.test_svd_transform_keeps_the_output,
 ]
 
 

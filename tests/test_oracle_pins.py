@@ -401,3 +401,47 @@ def test_ffn_gate_and_up_use_their_own_norms():
     assert r["idx_up"].tolist() == [2, 3]
     # gate and up outputs never overlap here, so h = 0 everywhere
     assert not r["h"].any()
+
+
+# ------------------------------------------------------------------------------------
+# the column-orthogonalising transform ([WINA] section 五)
+# ------------------------------------------------------------------------------------
+
+
+def test_svd_transform_orthogonal_columns_and_norms():
+    rng = np.random.default_rng(31)
+    W = rng.standard_normal((40, 16)) * rng.lognormal(0.0, 0.5, size=16)  # correlated scales
+    Wp, V = O.svd_transform(W)
+    s = np.linalg.svd(W, compute_uv=False)
+    G = Wp.T @ Wp
+    off = G - np.diag(np.diag(G))
+    assert np.abs(off).max() <= 1e-10 * s[0] ** 2
+    assert np.allclose(np.diag(G), s**2, rtol=1e-10)
+    assert np.allclose(V.T @ V, np.eye(16), atol=1e-12)  # V is orthogonal
+    # the gate's column norms of W' are the singular values (one rounding to float32)
+    assert np.allclose(O.col_norms(Wp), s.astype(np.float32), rtol=1e-6)
+
+
+def test_svd_transform_keeps_the_output():
+    rng = np.random.default_rng(32)
+    W = rng.standard_normal((30, 12))
+    x = rng.laplace(size=12)
+    Wp, V = O.svd_transform(W)
+    y = O.dense_matvec(W, x)
+    assert np.allclose(O.dense_matvec(Wp, V.T @ x), y, rtol=1e-12, atol=1e-12 * np.abs(y).max())
+
+
+def test_svd_transform_makes_wina_the_error_minimiser():
+    # on a non-orthogonal W the WINA set need not minimise the output error; after the
+    # transform (gate on W' and x' = V^T x) it does, for every K (brute force, n = 8)
+    rng = np.random.default_rng(33)
+    for trial in range(10):
+        W = rng.standard_normal((12, 8)) @ rng.standard_normal((8, 8))  # correlated columns
+        Wp, V = O.svd_transform(W)
+        xp = V.T @ rng.laplace(size=8)
+        c = O.col_norms(Wp)
+        for k in range(0, 9):
+            errs = {comb: O.output_error(Wp, xp, list(comb)) for comb in itertools.combinations(range(8), k)}
+            best = min(errs.values())
+            wina = tuple(O.wina_select(xp.astype(np.float32), c, k).tolist())
+            assert errs[wina] <= best * (1 + 1e-6) + 1e-12, (trial, k)
