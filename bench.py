@@ -120,9 +120,15 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------
 
 
-def oracle_sample(p: float, budget_s: float = 12.0, max_tokens: int = 20) -> dict:
+def oracle_sample(p: float, budget_s: float = 12.0, max_tokens: int = 20, threads: int | None = None) -> dict:
     """Time the CPU oracle's per-token FFN (select + float64 products) on one layer of
-    the same workload, as many tokens as fit in about budget_s seconds."""
+    the same workload, as many tokens as fit in about budget_s seconds; with `threads`,
+    the BLAS thread pools are limited to that many threads for the run."""
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+
+        with threadpool_limits(limits=threads):
+            return oracle_sample(p, budget_s, max_tokens)
     import oracle as O
 
     try:
@@ -419,9 +425,12 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = oracle_sample(args.p)
+        r1 = oracle_sample(args.p, budget_s=8.0, max_tokens=5, threads=1)
         line["cpu_baseline"] = {"value": r["gbs"], "unit": "GB/s", "us_per_layer": r["us_per_layer"],
                                 "cores": r["cores"], "kind": "oracle",
-                                "sample": f"{r['tokens']} tokens through one layer (median per token)"}
+                                "sample": f"{r['tokens']} tokens through one layer (median per token)",
+                                "one_thread": {"value": r1["gbs"], "us_per_layer": r1["us_per_layer"],
+                                               "sample": f"{r1['tokens']} tokens, BLAS limited to one thread"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
