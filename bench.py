@@ -159,6 +159,91 @@ def oracle_sample(p: float, budget_s: float = 12.0, max_tokens: int = 20, thread
 # ------------------------------------------------------------------------------------
 
 
+def _events(torch, stream, fn, steps: int) -> float:
+    """ms of `steps` calls of fn, CUDA events on `stream` (synchronised on both sides)."""
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def measure_spark_ffn(W, torch, stream, steps: int, copies: int = 4) -> dict:
+    """Gemma-2-2B FFN (d 2304, ffn 9216, bf16) with the Spark statistical gate (keep
+    fraction 0.08) on every projection, one token per call, `copies` distinct weight
+    copies (4 x 127 MB, above L2) called in turn. Bytes: the kept rows (read back from
+    the call's kept-set views) plus the vectors."""
+    cfg = synth.make_gemma2_2b_spark(batch=1)
+    d, ffn, s = cfg["d"], cfg["ffn"], cfg["s"]
+    fs = []
+    for _ in range(copies):
+        up = [torch.from_numpy(cfg[k].view(np.int16)).cuda().view(torch.bfloat16) for k in ("Wg", "Wu", "Wd")]
+        fs.append(W.ffn_prepare(*up))
+        del up
+    x = torch.from_numpy(cfg["x_bf16"].view(np.int16)).cuda().view(torch.bfloat16)
+    ws = W.Workspace(W.OP_FFN_SWIGLU, d, ffn, 0, 1)
+    y = torch.empty((1, d), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step():
+        for f in fs:
+            W.sparse_ffn_swiglu(f, x, W.GATE_STAT, s=s, ws=ws, status=st, y=y)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())}")
+    v = W.ffn_ws_view(ws, d, ffn, 1)
+    kg, ku, kd = (int(v[k].sum().item()) for k in ("keep_gate", "keep_up", "keep_down"))
+    nbytes = (kg + ku) * ffn * 2 + kd * d * 2 + d * 2 + d * 4
+    ms = _events(torch, stream, step, steps)
+    us = ms / (steps * copies) * 1e3
+    return {"us_per_layer": us, "effective_gbs": nbytes / (us * 1e-6) / 1e9, "bytes_per_layer": nbytes,
+            "kept": [kg, ku, kd], "gate": "Spark statistical top-k, s = 0.08", "path": "fused kernel, eager calls"}
+
+
+def measure_ultrasparse(W, torch, stream, steps: int, copies: int = 2) -> dict:
+    """Down projection 14336 -> 4096 (bf16), 256 tokens with 143 nonzero inputs each: the
+    nonzero set selected on the GPU and the sparse product, per step; `copies` distinct
+    weight copies (2 x 117 MB) called in turn. Bytes: the union of the tokens' columns
+    (read once by a union product) plus the inputs and outputs."""
+    cfg = synth.make_ultrasparse_down()
+    n, m, nnz = cfg["n"], cfg["m"], cfg["nnz"]
+    Wts = []
+    for _ in range(copies):
+        Wd = torch.from_numpy(cfg["W"].view(np.int16)).cuda().view(torch.bfloat16)
+        Wts.append(W.pack_in_major(Wd))
+        del Wd
+    xb = torch.from_numpy(cfg["x"].view(np.int16)).cuda().view(torch.bfloat16)
+    B = xb.shape[0]
+    ws = W.Workspace(W.OP_SPARSE_MATVEC, n, m, nnz, B)
+    y = torch.empty((B, m), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step():
+        for Wt in Wts:
+            idx, xs = W.select_topk(xb, None, nnz)
+            W.sparse_matvec(Wt, idx, xs, ws=ws, status=st, y=y)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())}")
+    idx, _ = W.select_topk(xb, None, nnz)
+    union = int(torch.unique(idx).numel())
+    nbytes = union * m * 2 + B * n * 2 + B * m * 4
+    ms = _events(torch, stream, step, steps)
+    us = ms / (steps * copies) * 1e3
+    return {"us_per_call": us, "effective_gbs": nbytes / (us * 1e-6) / 1e9, "union_columns": union,
+            "bytes_per_call": nbytes, "tensor_pipe": "not used (per-token CUDA-core products)",
+            "path": "wina_select_topk (nonzero set) + sparse_matvec, eager calls"}
+
+
 def reduce_max(v: float, world: int, device: str) -> float:
     """The maximum of v over the ranks of the default process group (every rank must
     call it; a single process returns v). Times are taken as the max over ranks."""
@@ -395,6 +480,18 @@ def main():
     e2e_ms = max_over_ranks(t_e0.elapsed_time(t_e1))
     e2e_gbs = world * nbytes * L * args.steps / (e2e_ms * 1e-3) / 1e9
 
+    # the other configurations of the scope table, measured on the same GPU (each guarded:
+    # a failure is reported in its entry and never affects the headline line)
+    extra = {}
+    try:
+        extra["spark_ffn_gemma2_2b_bs1"] = measure_spark_ffn(W, torch, stream, max(3, args.steps // 2))
+    except Exception as e:  # pragma: no cover - reported, not raised
+        extra["spark_ffn_gemma2_2b_bs1"] = {"error": f"{type(e).__name__}: {e}"}
+    try:
+        extra["ultrasparse_down_b256"] = measure_ultrasparse(W, torch, stream, max(3, args.steps // 2))
+    except Exception as e:  # pragma: no cover
+        extra["ultrasparse_down_b256"] = {"error": f"{type(e).__name__}: {e}"}
+
     peak, peak_kind = _peaks()
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
     traffic = None  # ncu dram bytes of one launch, valid only for the kernel it was taken on
@@ -418,6 +515,7 @@ def main():
                   "kernel_us_events": eager_kern_ms * 1e3},
         "dense": {"us_per_layer": us_layer_dense, "speedup": us_layer_dense / us_layer},
         "batched": batched,
+        "other_configs": extra,
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "us_per_layer": e2e_ms / args.steps * 1e3 / L,
                 "h2d_bytes_per_step": L * D * 2, "d2h_bytes_per_step": L * D * 4},
         "gpu_launches": L * args.steps,
