@@ -81,6 +81,32 @@ def _silu_minus(g):
         return g / (1.0 + np.exp(g))
 
 
+def _ffn_stat_variant(abs_x=False, up_from_xc=False, h64=False):
+    """A copy of the oracle's FFN whose Spark (stat) branch carries one planted mistake:
+    gate/up thresholding |x|, the up set taken from x * c_up, or the down gate on the
+    float64 h instead of the float32 h held between the projections."""
+    real = W.ffn_swiglu
+
+    def ffn(Wg, Wu, Wd, cg, cu, cd, x, kg, ku, kd, mode="topk", s=0.08):
+        if mode != "stat":
+            return real(Wg, Wu, Wd, cg, cu, cd, x, kg, ku, kd, mode=mode, s=s)
+        x = np.asarray(x)
+        xv = np.abs(x) if abs_x else x
+        ig = W.spark_threshold(xv, s)["idx"]
+        iu = W.spark_threshold(np.asarray(x, dtype=np.float32) * np.asarray(cu, dtype=np.float32), s)["idx"] \
+            if up_from_xc else ig
+        x64 = np.asarray(x, dtype=np.float64)
+        g = W.sparse_matvec(Wg, ig, x64[ig])
+        u = W.sparse_matvec(Wu, iu, x64[iu])
+        h = W.silu(g) * u
+        h32 = h.astype(np.float32)
+        idn = W.spark_threshold(h if h64 else h32, s)["idx"]
+        y = W.sparse_matvec(Wd, idn, h[idn])
+        return dict(idx_gate=ig, idx_up=iu, g=g, u=u, h=h, h32=h32, idx_down=idn, y=y)
+
+    return ffn
+
+
 def _svd_transposed(Wm):
     # transposed operand: W V^T instead of W V
     W64 = np.asarray(Wm, dtype=np.float64)
@@ -99,6 +125,9 @@ MUTATIONS = {
     "spark:wrong-tail": ("spark_threshold", _spark_wrong_tail),
     "silu:sign": ("silu", _silu_minus),
     "svd_transform:transposed-V": ("svd_transform", _svd_transposed),
+    "ffn_swiglu:stat-gate-on-abs-x": ("ffn_swiglu", _ffn_stat_variant(abs_x=True)),
+    "ffn_swiglu:stat-up-set-from-x-times-c": ("ffn_swiglu", _ffn_stat_variant(up_from_xc=True)),
+    "ffn_swiglu:stat-down-gate-on-float64-h": ("ffn_swiglu", _ffn_stat_variant(h64=True)),
 }
 
 PINS = [
@@ -110,6 +139,7 @@ PINS = [
     P.test_sparse_matvec_uses_columns_not_rows,
     P.test_silu_closed_forms,
     P.test_ffn_identity_weights_hand_computed,
+    P.test_golden_spark_ffn_example,
     P.test_gate_scores_single_fp32_multiply,
     lambda: P.test_spark_keep_fraction_gaussian(2304, 2e-3, 0.03),
     P.test_svd_transform_orthogonal_columns_and_norms,

@@ -390,6 +390,50 @@ def test_ffn_identity_weights_hand_computed():
     assert np.allclose(r["y"], (xd / (1 + np.exp(-xd))) * xd, rtol=1e-15, atol=0)
 
 
+def _zstar_exact(v, i):
+    """(v_i - mean) / std of v in exact rational arithmetic, square root to 60 digits."""
+    from decimal import Decimal, localcontext
+
+    fv = [Fraction(float(a)) for a in v]
+    n = len(fv)
+    mu = sum(fv) / n
+    var = sum((a - mu) ** 2 for a in fv) / n
+    with localcontext() as ctx:
+        ctx.prec = 60
+        num = Decimal((fv[i] - mu).numerator) / Decimal((fv[i] - mu).denominator)
+        return num / (Decimal(var.numerator) / Decimal(var.denominator)).sqrt()
+
+
+def test_golden_spark_ffn_example():
+    # Spark gate on every projection of a SwiGLU FFN with identity weights: gate and up
+    # share the set of the signed x, the down gate thresholds the float32 h
+    g = _read_golden("spark_ffn_worked_example.txt")
+    eye = np.eye(6)
+    x = np.array(g["x"], dtype=np.float32)
+    assert float(x[4]) == 41.0 + 2.0 ** -18
+    cg = np.ones(6, dtype=np.float32)
+    cu = np.array(g["c_up"], dtype=np.float32)
+    cd = np.ones(6, dtype=np.float32)
+    s = g["s"][0]
+    # the knife edge, independently of the oracle: the stdlib quantile of 1 - s lies
+    # strictly between the exact cut points of the float64 and the float32 h4
+    from decimal import Decimal
+
+    z = Decimal(NormalDist().inv_cdf(1.0 - s))
+    h64 = [0.0, 0.0, 0.0, 0.0, (41.0 + 2.0 ** -18) ** 2, 2500.0]
+    h32 = [float(np.float32(a)) for a in h64]
+    assert h32[4] == g["h4_float32"][0] and h64[4] == g["y"][4]
+    z32, z64 = _zstar_exact(h32, 4), _zstar_exact(h64, 4)
+    assert abs(z32 - Decimal(g["zstar_float32"][0])) < Decimal("1e-15")
+    assert abs(z64 - Decimal(g["zstar_float64"][0])) < Decimal("1e-15")
+    assert z64 < z < z32
+    r = O.ffn_swiglu(eye, eye, eye, cg, cu, cd, x, 0, 0, 0, mode="stat", s=s)
+    assert r["idx_gate"].tolist() == [int(v) for v in g["keep_gate"]]
+    assert r["idx_up"].tolist() == [int(v) for v in g["keep_up"]]
+    assert r["idx_down"].tolist() == [int(v) for v in g["keep_down"]]
+    assert r["y"].tolist() == g["y"]
+
+
 def test_ffn_gate_and_up_use_their_own_norms():
     # gate and up see the same x but different c: their kept sets must differ
     x = np.array([1.0, 1.0, 1.0, 1.0], dtype=np.float32)
