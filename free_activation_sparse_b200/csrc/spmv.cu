@@ -241,7 +241,6 @@ extern "C" wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt,
   const int epv = wdt == WINA_BF16 ? 8 : 4;
   if (n < 1 || n > INT32_MAX || m < epv || m % epv != 0 || m / epv > (int64_t)kNT * 8) return WINA_ERR_INVALID_ARG;
   if (batch < 1 || batch > INT32_MAX || ld_idx < 0 || ld_idx > INT32_MAX) return WINA_ERR_INVALID_ARG;
-  if (batch * m > kNoAllocMaxOutputs) return WINA_ERR_INVALID_ARG;  // the fixed scratch is too small
   if (k < -1 || k > ld_idx || (k == -1 && !count)) return WINA_ERR_INVALID_ARG;
   if (!Wt || !y || (ld_idx > 0 && (!idx || !xs))) return WINA_ERR_INVALID_ARG;
   if (!aligned(Wt, 16) || !aligned(y, 16) || (idx && !aligned(idx, 4)) || (xs && !aligned(xs, 4)) ||
@@ -256,12 +255,18 @@ extern "C" wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt,
                         : max_coresident_grid(k_sparse_matvec<false>, kNT, smem);
   if (gmax < 1) return WINA_ERR_CUDA;
   const int B = (int)batch;
+  // With at least one co-resident CTA per token (P == 1) every CTA writes its token's y
+  // directly and the scratch is not used, whatever the size. Otherwise the split-K
+  // partial rows must fit in the fixed array: at least two per token.
+  if (B < gmax && batch * m > kNoAllocMaxOutputs) return WINA_ERR_INVALID_ARG;
   int P = B < gmax ? gmax / B : 1;
   const int kmax = k >= 0 ? (int)k : (int)ld_idx;
   const int want = (kmax + 7) / 8;
   if (P > want) P = want > 0 ? want : 1;
-  const int64_t fit = kNoAllocPartialFloats / (batch * m);  // partial rows per token that fit
-  if (P > fit) P = (int)fit;                                // >= 2 by the size check above
+  if (P > 1) {
+    const int64_t fit = kNoAllocPartialFloats / (batch * m);  // partial rows per token that fit
+    if (P > fit) P = (int)fit;                                // >= 2 by the size check above
+  }
   // The barrier words must start at zero: clear them on the stream (the partial rows
   // are always written before they are read). Calls that overlap on the GPU share this
   // scratch and race.

@@ -201,9 +201,11 @@ wina_status_t stat_topk_threshold(const void* v, wina_dtype_t vdt, int64_t n, do
 
 /* Sparse product over the kept channels ("Spark Transformer", section 3.1, SVMM):
  *   y[b][:] = sum over r < k_b of xs[b][r] * Wt[idx[b][r]][:]      for b < batch,
- * reading only the kept rows of the input-major weight. One token (batch == 1) is
- * split across all SMs by kept rows (split-K) with a deterministic reduction; several
- * tokens are served from the union of their kept rows, each row read once per call.
+ * reading only the kept rows of the input-major weight. The co-resident grid is shared
+ * among the tokens: token b gets P = grid / batch CTAs (at least one), which split its
+ * kept rows (split-K) and, when P > 1, sum their partial rows in a fixed order after a
+ * grid barrier, so results are bit-reproducible. Each token reads its own kept rows: a
+ * row kept by several tokens is read once per token.
  *   Wt:    device [n][m] of wdt (m % 8 == 0 and m <= 32768 for bf16; m % 4 == 0 and
  *          m <= 16384 for f32).
  *   idx:   device int32 [batch][ld_idx]: kept input channels of each token (any order;
@@ -228,10 +230,15 @@ wina_status_t sparse_matvec(const void* Wt, wina_dtype_t wdt, int64_t n, int64_t
  * the scratch (a barrier word pair and the split-K partial rows) lives in a fixed
  * 8 MiB + 256 B array of device memory declared by the library, which every GPU that
  * loads the library holds until the process exits. It allocates nothing.
- *   Limit: batch * m <= 1,048,576 (at least two partial rows per token must fit in
- *   the 2^21-float array); larger calls return WINA_ERR_INVALID_ARG.
+ *   Limit: when batch is smaller than the co-resident grid (148 CTAs on a B200), a
+ *   token is split over several CTAs whose partial rows live in the 2^21-float array,
+ *   so batch * m <= 1,048,576 is required (at least two partial rows per token);
+ *   larger calls return WINA_ERR_INVALID_ARG. With batch at least the grid, each
+ *   token has its own CTA, the array is not used and any size is accepted.
  *   The first call on a device looks up the array's device address (once per device,
- *   with that device current); make that first call before any stream capture.
+ *   with that device current) and keeps it for the life of the process; make that
+ *   first call before any stream capture, and do not use this entry point on a device
+ *   after cudaDeviceReset (the kept address would be stale).
  *   Every call clears the barrier words on `stream` and then reuses the same array:
  *   calls that overlap on the GPU (other streams, other threads) race and must not
  *   be issued. */
