@@ -542,7 +542,7 @@ def main():
         "dtype": "bf16 weights, f32 accumulate", "data": "synthetic", "config": config,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
-                     "kernel": "k_ffn_fused (one launch per layer)", "bytes_per_launch": nbytes,
+                     "kernel": "k_ffn_decode (one launch per layer)", "bytes_per_launch": nbytes,
                      "kernel_us": kern_ms * 1e3, "timing": "CUDA graph of the L-layer step, events around K replays"},
         "eager": {"us_per_layer": eager_ms / max(3, args.steps // 2) * 1e3 / L,
                   "kernel_us_events": eager_kern_ms * 1e3},
@@ -571,7 +571,7 @@ def main():
 def _kernel_sha() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("common.cuh", "ffn.cu"):
+    for f in ("common.cuh", "ffn_decode.cu"):
         with open(os.path.join(ROOT, "free_activation_sparse_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

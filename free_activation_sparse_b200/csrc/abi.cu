@@ -31,6 +31,8 @@ OccEntry g_occ[kCacheSlots];
 int g_nocc = 0;
 SmemEntry g_smem[kCacheSlots];
 int g_nsmem = 0;
+SmemEntry g_l1[kCacheSlots];
+int g_nl1 = 0;
 }  // namespace
 
 int device_sm_count() {
@@ -67,6 +69,22 @@ cudaError_t ensure_smem_limit(const void* kern, size_t smem) {
       return cudaSuccess;
     }
   if (g_nsmem < kCacheSlots) g_smem[g_nsmem++] = SmemEntry{dev, kern, smem};
+  return cudaSuccess;
+}
+
+cudaError_t ensure_prefer_l1(const void* kern) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (int i = 0; i < g_nl1; ++i)
+      if (g_l1[i].dev == dev && g_l1[i].kern == kern) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxL1);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_nl1 < kCacheSlots) g_l1[g_nl1++] = SmemEntry{dev, kern, 0};
   return cudaSuccess;
 }
 

@@ -405,194 +405,6 @@ __device__ void hist_crossing(const uint32_t* __restrict__ hist, uint32_t r, uin
   *cnt = s_cnt;
 }
 
-// Exact top-K of keys[0..n) in SMEM (ties to the lower index) as a kept-channel
-// bitmask, in two parts so that a caller can run the second part on a subset of its
-// warps:
-//   radix_crossing  (every thread of the block) finds the boundary bin B, given hist =
-//                   the counts of the keys' top 12 bits (key >> 19; bit 31 of a
-//                   non-negative float is 0), filled while the keys were produced;
-//   radix_finish    (threads [0, NT), synchronised by sync()) sets the flags.
-// Keys above B are kept. The bin's keys are listed and their next 8 bits counted in a
-// 256-bin histogram; one warp finds the sub-bin B2 holding the K-th key; keys above B2
-// are kept and the few keys in B2 are ranked exactly. A bin with more than kSelCand
-// keys is left to the general search (select_threshold). flags[w] bit l = channel
-// 32w + l is kept. SMEM: keys 16-byte aligned and readable up to the next multiple of
-// 128 entries (the excess is ignored), hist [kSelBins + 256] (the first kSelBins
-// filled, the last 256 zero), cand [2 * kSelCand], red [>= 2 * NT/32 + 8].
-
-struct Crossing {
-  int bin;         // boundary bin B (12-bit digit)
-  uint32_t above;  // keys in higher bins
-  uint32_t cnt;    // keys in B
-};
-
-template <int NT>
-__device__ Crossing radix_crossing(const uint32_t* __restrict__ hist, int K, uint32_t* red) {
-  static_assert(kSelBins == 4096, "12-bit digit");
-  __syncthreads();  // the caller's histogram updates are complete
-  Crossing c;
-  hist_crossing<NT>(hist, (uint32_t)K, red, &c.bin, &c.above, &c.cnt);
-  return c;
-}
-
-template <int NT, typename Sync>
-__device__ void radix_finish(const uint32_t* __restrict__ keys, int n, int K, Crossing cr,
-                             uint32_t* __restrict__ hist, uint32_t* __restrict__ cand, uint32_t* __restrict__ flags,
-                             Sync sync, long long* st = nullptr) {
-  constexpr int NW = NT / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = (n + 31) / 32;
-  const int B = cr.bin;
-  const uint32_t r = (uint32_t)K - cr.above;  // kept among the bin's keys
-  const uint32_t nb = cr.cnt;                 // keys in the bin (<= kSelCand)
-  uint32_t* list = hist;                      // the bin's (key, channel) pairs
-  uint32_t* sub = hist + kSelBins;            // counts of their next 8 bits (zeroed by the caller)
-  __shared__ uint32_t s_n, s_b2, s_above2, s_nties;
-  if (threadIdx.x == 0) {
-    s_n = 0u;
-    s_nties = 0u;
-  }
-  sync();
-  // 1. one pass over the keys: flags of the channels above B; the bin's keys listed
-  //    (one list slot range per warp step) and counted by their next 8 bits. Each lane
-  //    takes four consecutive channels (one 16-byte load); eight lanes' nibbles are
-  //    merged into a flag word by shuffles.
-  const int n128 = (n + 127) / 128;
-  for (int q = warp; q < n128; q += NW) {
-    const int j0 = q * 128 + lane * 4;
-    const uint4 k4 = reinterpret_cast<const uint4*>(keys)[q * 32 + lane];
-    const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
-    uint32_t above_nib = 0u, inb[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int bj = j0 + e < n ? (int)(kk[e] >> 19) : -1;
-      above_nib |= bj > B ? (1u << e) : 0u;
-      inb[e] = __ballot_sync(0xffffffffu, bj == B);
-    }
-    uint32_t fa = above_nib << (4 * (lane & 7));
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) fa |= __shfl_xor_sync(0xffffffffu, fa, o);
-    const int w = q * 4 + (lane >> 3);
-    if ((lane & 7) == 0 && w < nw) flags[w] = fa;
-    const uint32_t tot = __popc(inb[0]) + __popc(inb[1]) + __popc(inb[2]) + __popc(inb[3]);
-    if (tot) {  // uniform across the warp
-      const uint32_t lt = (1u << lane) - 1u;
-      uint32_t at = 0u;
-      if (lane == 0) at = atomicAdd(&s_n, tot);
-      at = __shfl_sync(0xffffffffu, at, 0) + __popc(inb[0] & lt) + __popc(inb[1] & lt) + __popc(inb[2] & lt) +
-           __popc(inb[3] & lt);
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if ((inb[e] >> lane) & 1u) {
-          list[2 * at] = kk[e];
-          list[2 * at + 1] = (uint32_t)(j0 + e);
-          atomicAdd(&sub[(kk[e] >> 11) & 255u], 1u);
-          ++at;
-        }
-    }
-  }
-  sync();
-  if (st && threadIdx.x == 0) st[1] = clock64();
-  // 2. warp 0 finds the sub-bin B2 holding the r-th largest of the bin's keys
-  if (warp == 0) {
-    uint32_t v[8], t = 0u;  // lane l: sub-bins 255 - 8l, ..., 248 - 8l (from the top)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      v[e] = sub[255 - 8 * lane - e];
-      t += v[e];
-    }
-    uint32_t x = t;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    uint32_t ab = x - t;  // keys in sub-bins above this lane's
-    const bool hit = ab < r && ab + t >= r;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      if (hit && ab < r && ab + v[e] >= r) {
-        s_b2 = (uint32_t)(255 - 8 * lane - e);
-        s_above2 = ab;
-      }
-      ab += v[e];
-    }
-  }
-  sync();
-  // 3. keys above B2 are kept; those in B2 go to a short list
-  const uint32_t B2 = s_b2, r2 = r - s_above2;
-  for (uint32_t e = threadIdx.x; e < nb; e += NT) {
-    const uint32_t k = list[2 * e], ch = list[2 * e + 1], sb = (k >> 11) & 255u;
-    if (sb > B2) {
-      atomicOr(&flags[ch >> 5], 1u << (ch & 31));
-    } else if (sb == B2) {
-      const uint32_t at = atomicAdd(&s_nties, 1u);
-      cand[2 * at] = k;
-      cand[2 * at + 1] = ch;
-    }
-  }
-  sync();
-  // 4. the r2 highest of that list (ties to the lower channel) are kept
-  const uint32_t nt = s_nties;
-  for (uint32_t c = threadIdx.x; c < nt; c += NT) {
-    const uint32_t kc = cand[2 * c], ic = cand[2 * c + 1];
-    uint32_t a = 0u;
-    for (uint32_t o = 0; o < nt; ++o) {
-      const uint32_t ko = cand[2 * o], io = cand[2 * o + 1];
-      a += (ko > kc || (ko == kc && io < ic)) ? 1u : 0u;
-    }
-    if (a < r2) atomicOr(&flags[ic >> 5], 1u << (ic & 31));
-  }
-  sync();
-}
-
-// Flags of the exact top-K (0 < K < n) by the general search (select_threshold), for
-// a boundary bin too full to rank. Every thread of the block must call it.
-template <int NT>
-__device__ void select_general_flags(const uint32_t* __restrict__ keys, int n, int K, uint32_t* __restrict__ hist,
-                                     uint32_t* __restrict__ cand, uint32_t* __restrict__ red,
-                                     uint32_t* __restrict__ flags) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = (n + 31) / 32;
-  const Threshold t = select_threshold<NT>(keys, n, K, hist, cand, red);
-  for (int w = warp; w < nw; w += NT / 32) {
-    const int j = w * 32 + lane;
-    const uint32_t bits = __ballot_sync(0xffffffffu, j < n && kept_by(t, keys[j], j));
-    if (lane == 0) flags[w] = bits;
-  }
-  __syncthreads();
-}
-
-// Both parts on the whole block (every thread must call it); K <= 0 and K >= n keep
-// nothing / everything, a boundary bin over kSelCand keys takes the general search.
-struct BlockSync {
-  __device__ void operator()() const { __syncthreads(); }
-};
-
-template <int NT>
-__device__ void select_topk_flags_radix(const uint32_t* __restrict__ keys, int n, int K, uint32_t* __restrict__ hist,
-                                        uint32_t* __restrict__ cand, uint32_t* __restrict__ red,
-                                        uint32_t* __restrict__ flags, long long* st = nullptr) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = (n + 31) / 32;
-  if (K <= 0 || K >= n) {
-    const int keep = K <= 0 ? 0 : n;
-    for (int w = threadIdx.x; w < nw; w += NT) {
-      const int rem = keep - w * 32;
-      flags[w] = rem >= 32 ? 0xffffffffu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
-    }
-    __syncthreads();
-    return;
-  }
-  const Crossing cr = radix_crossing<NT>(hist, K, red);
-  if (st && threadIdx.x == 0) st[0] = clock64();
-  if (cr.cnt > (uint32_t)kSelCand) {
-    select_general_flags<NT>(keys, n, K, hist, cand, red, flags);
-    return;
-  }
-  radix_finish<NT>(keys, n, K, cr, hist, cand, flags, BlockSync{}, st);
-}
-
 // ------------------------------------------------------------------------------------
 // one-pass mean / variance (Welford per thread, Chan's pairwise merge across threads)
 // ------------------------------------------------------------------------------------

@@ -1,0 +1,800 @@
+// Single-token SwiGLU FFN decode with the gate on every projection ("WAS" article, core
+// innovations: the gate is applied per component, gate/up/down among them; "WINA"
+// article, section 一: each projection scores with the column norms of its own weight and
+// keeps its own K; "Spark Transformer", section 2.2: the statistical threshold variant).
+//
+// One persistent cooperative launch, one CTA of 1024 threads per SM, little shared
+// memory, so that most of each SM's L1 is free to hold the weight loads in flight:
+//   A  CTAs [0, Gg) take the gate projection, the rest up. Every CTA scores x against its
+//      projection's c with the keys held in registers (thread t owns channels
+//      t, t + 1024, ...), finds the kept set by a radix select on the float32 key bits
+//      (histogram of the top 12 bits, then 8, 8 and 3 bits only while needed; equal keys
+//      resolved by index), and lists the kept channels whose rank r in ascending channel
+//      order satisfies r mod parts == its part: the kept rows are dealt out round robin,
+//      so at any moment all SMs read rows from the same neighbourhood of the weight.
+//   B  The CTA streams its rows with 16-byte read-only loads (several rows in flight per
+//      thread), accumulates x_j * row_j in float32 registers and stores its partial row
+//      of g or u (plain stores: float atomics from every SM onto the same addresses
+//      serialise in L2 for microseconds).
+//   -- grid barrier --
+//   C1 CTA b sums its slice of the channels over all partial rows in a fixed order and
+//      writes h = silu(g) * u and the down scores |h * c_down| for that slice.
+//   -- grid barrier --
+//   C2 Every CTA loads all down scores into registers, selects and lists its share of
+//      the down rows the same way.
+//   E  Streams them into its partial row of y.
+//   -- grid barrier --
+//   E2 CTA b sums its slice of y over the partial rows in a fixed order.
+// Every wait is a grid barrier with a time limit. Selections are exact and identical on
+// every CTA, and every sum is taken in a fixed order, so the results are bit-reproducible.
+#include <math.h>
+
+#include <algorithm>
+
+#include "internal.h"
+
+namespace wina {
+
+constexpr int kDT = 1024;       // threads per CTA
+constexpr int kDW = kDT / 32;   // warps per CTA
+constexpr int kDKeys = 16;      // channels per thread at most (vectors of up to 16384)
+constexpr int kDMaxN = kDT * kDKeys;
+
+struct DecodeParams {
+  const void* wt_gate;
+  const void* wt_up;
+  const void* wt_down;
+  const float* c_gate;
+  const float* c_up;
+  const float* c_down;
+  const void* x;
+  int xdt;
+  int d, ffn;
+  int mode;
+  int k_gate, k_up, k_down;
+  double z;
+  float* y;
+  int Gg;        // CTAs on the gate projection
+  int list_cap;  // rows per CTA list
+  uint32_t sm_flags, sm_wpre, sm_lrow, sm_lval;  // SMEM offsets (the histogram is at 0)
+  GridBarrier* bar;
+  float* part;      // [G][pstride] float32 partial rows (g / u in phase B, y in phase E)
+  int pstride;      // floats per partial row (>= max(d, ffn), a multiple of 4)
+  uint32_t* dkeys;  // [ffn] down-gate scores (float32 bits), written in slices in C1
+  float* h;
+  uint8_t* keep_g;
+  uint8_t* keep_u;
+  uint8_t* keep_d;
+  long long* stamps;
+  unsigned long long* cta_t;
+  int32_t* status;
+};
+
+// Dynamic SMEM: hist [kSelBins + 256] | flags [nw] | word prefix [nw] | list rows [cap] |
+// list values [cap] | group reduction [red_floats] (overlays hist).
+struct DecodeSmem {
+  uint32_t hist, flags, wpre, lrow, lval, total;
+};
+
+__host__ __device__ inline DecodeSmem decode_smem(int n_max, int cap, int red_floats) {
+  DecodeSmem L;
+  const uint32_t nw = (uint32_t)(n_max + 31) / 32;
+  const uint32_t hist_bytes = (uint32_t)(kSelBins + 256) * 4u;
+  const uint32_t red_bytes = (uint32_t)red_floats * 4u;
+  uint32_t o = 0;
+  L.hist = o;
+  o += (hist_bytes > red_bytes ? hist_bytes : red_bytes);
+  o = (o + 15u) & ~15u;
+  L.flags = o;
+  o += nw * 4u;
+  o = (o + 15u) & ~15u;
+  L.wpre = o;
+  o += nw * 4u;
+  o = (o + 15u) & ~15u;
+  L.lrow = o;
+  o += (uint32_t)cap * 4u;
+  o = (o + 15u) & ~15u;
+  L.lval = o;
+  o += (uint32_t)cap * 4u;
+  L.total = (o + 127u) & ~127u;
+  return L;
+}
+
+// Threads per row and row groups of a row of V 16-byte vectors: rows of more than 256
+// vectors take 512 threads (two groups), shorter rows a power of two >= V.
+__host__ __device__ inline int decode_tpr(int V) {
+  int t = 32;
+  while (t < V && t < kDT / 2) t <<= 1;
+  return t;
+}
+
+__device__ __forceinline__ float silu_d(float g) { return g / (1.0f + expf(-g)); }
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void dstamp(long long* s, int i) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) s[i] = clock64();
+}
+__device__ __forceinline__ void dcta_time(unsigned long long* t, int i) {
+  if (threadIdx.x == 0) t[blockIdx.x * 4 + i] = globaltimer_ns();
+}
+
+// ------------------------------------------------------------------------------------
+// selection with the keys in registers
+// ------------------------------------------------------------------------------------
+
+// Bin holding the r-th largest of `nb` counts (nb <= 256), from the top: one warp, each
+// lane summing nb/32 consecutive bins. Writes bin, count above, the bin's count.
+__device__ __forceinline__ void small_crossing(const uint32_t* h, int nb, uint32_t r, uint32_t* out3) {
+  const int lane = threadIdx.x & 31;
+  const int per = nb / 32;  // 8 for 256 bins; nb >= 32 and a multiple of 32
+  uint32_t v[8], t = 0u;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    v[e] = e < per ? h[nb - 1 - per * lane - e] : 0u;
+    t += v[e];
+  }
+  uint32_t x = t;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  uint32_t ab = x - t;
+  const bool hit = ab < r && ab + t >= r;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    if (hit && e < per && ab < r && ab + v[e] >= r) {
+      out3[0] = (uint32_t)(nb - 1 - per * lane - e);
+      out3[1] = ab;
+      out3[2] = v[e];
+    }
+    ab += v[e];
+  }
+}
+
+// Exact top-K of the keys held in registers (thread t owns channels t + i * kDT, i < kpt,
+// those >= n absent), ties to the lower channel, as a threshold: kept(j) <=> key_j > T or
+// (key_j == T and j <= cut). Radix passes on bits 30..19, 18..11, 10..3 and 2..0 of the
+// keys, each restricted to the keys that share the prefix found so far, stop as soon as
+// every key of the crossing bin is kept. Every thread must call it. hist: SMEM of
+// kSelBins + 256 words, zero on entry (see clear_hist).
+template <int KMAX>
+__device__ __forceinline__ Threshold radix_select_regs(const uint32_t (&key)[KMAX], int kpt, int n, int K,
+                                                       uint32_t* hist) {
+  __shared__ uint32_t s_x[4];
+  __shared__ Threshold s_t;
+  __shared__ uint32_t s_cnt[kDW];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (K <= 0) return Threshold{0xffffffffu, -1};
+  if (K >= n) return Threshold{0u, n - 1};
+  uint32_t r = (uint32_t)K;
+  // pass 1: 12-bit digit (bit 31 of a non-negative float is 0); the caller zeroed hist
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i)
+    if (i < kpt && t + i * kDT < n) atomicAdd(&hist[key[i] >> 19], 1u);
+  __syncthreads();
+  {
+    int bin;
+    uint32_t above, cnt;
+    hist_crossing<kDT>(hist, r, s_cnt, &bin, &above, &cnt);  // ends with __syncthreads
+    r -= above;
+    uint32_t prefix = (uint32_t)bin;
+    int shift = 19;
+    if (r == cnt) return Threshold{prefix << shift, n - 1};  // every key of the bin is kept
+    // passes 2-4: bits 18..11, 10..3, 2..0
+#pragma unroll 1
+    for (int p = 0; p < 3; ++p) {
+      const int w = p < 2 ? 8 : 3;
+      const int nb = 1 << w;
+      const int nsh = shift - w;
+      uint32_t* sub = hist + kSelBins;
+      if (p > 0) {  // zeroed by the caller for the first of these passes
+        if (t < 256) sub[t] = 0u;
+        __syncthreads();
+      }
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i)
+        if (i < kpt && t + i * kDT < n && (key[i] >> shift) == prefix) atomicAdd(&sub[(key[i] >> nsh) & (nb - 1)], 1u);
+      __syncthreads();
+      if (warp == 0) {
+        if (nb >= 32) {
+          small_crossing(sub, nb, r, s_x);
+        } else {
+          // 8 bins: lane l < 8 holds bin 7 - l
+          const uint32_t v = lane < nb ? sub[nb - 1 - lane] : 0u;
+          uint32_t x = v;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
+          const uint32_t ab = x - v;
+          if (lane < nb && ab < r && ab + v >= r) {
+            s_x[0] = (uint32_t)(nb - 1 - lane);
+            s_x[1] = ab;
+            s_x[2] = v;
+          }
+        }
+      }
+      __syncthreads();
+      const uint32_t b2 = s_x[0], ab2 = s_x[1], c2 = s_x[2];
+      __syncthreads();
+      r -= ab2;
+      prefix = (prefix << w) | b2;
+      shift = nsh;
+      if (r == c2) return Threshold{prefix << shift, n - 1};
+    }
+    // all 31 bits resolved: the keys equal to T = prefix; keep the r lowest channels
+    const uint32_t T = prefix;
+    // counts of equal keys per register slot i (channels i*kDT .. i*kDT + kDT - 1)
+    int islot = 0;
+    uint32_t before = 0u;
+#pragma unroll 1
+    for (int i = 0; i < kpt; ++i) {
+      uint32_t ki = 0u;
+#pragma unroll
+      for (int q = 0; q < KMAX; ++q)
+        if (q == i) ki = key[q];
+      const int c = __syncthreads_count(t + i * kDT < n && ki == T);
+      if (before + (uint32_t)c >= r) {
+        islot = i;
+        break;
+      }
+      before += (uint32_t)c;
+    }
+    uint32_t ki = 0u;
+#pragma unroll
+    for (int q = 0; q < KMAX; ++q)
+      if (q == islot) ki = key[q];
+    const bool eq = t + islot * kDT < n && ki == T;
+    const uint32_t m = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) s_cnt[warp] = (uint32_t)__popc(m);
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t v = s_cnt[lane];
+      uint32_t x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      s_cnt[lane] = x - v;  // equal keys in lower warps
+    }
+    __syncthreads();
+    const uint32_t rr = r - before;  // the rr-th equal key of slot islot (1-based) is the cut
+    const uint32_t lower = s_cnt[warp] + (uint32_t)__popc(m & ((1u << lane) - 1u));
+    if (eq && lower + 1u == rr) s_t = Threshold{T, t + islot * kDT};
+    __syncthreads();
+    const Threshold res = s_t;
+    __syncthreads();
+    return res;
+  }
+}
+
+__device__ __forceinline__ void clear_hist(uint32_t* hist) {
+  for (int i = threadIdx.x; i < kSelBins + 256; i += kDT) hist[i] = 0u;
+}
+
+// Flags of a threshold over the register-held keys: bit l of word w = channel 32w + l.
+template <int KMAX>
+__device__ __forceinline__ void flags_from_keys(const uint32_t (&key)[KMAX], int kpt, int n, Threshold th,
+                                                uint32_t* flags) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    if (i < kpt) {
+      const int j = t + i * kDT;
+      const bool k = j < n && (key[i] > th.T || (key[i] == th.T && j <= th.cut));
+      const uint32_t bits = __ballot_sync(0xffffffffu, k);
+      const int w = i * kDW + warp;
+      if (lane == 0 && w < (n + 31) / 32) flags[w] = bits;
+    }
+  }
+}
+
+// Spark threshold on register-held values: mu + sigma * z, moments in float64
+// (Welford per thread, Chan's pairwise merge in a fixed order), strict v > t.
+template <int KMAX>
+__device__ __forceinline__ void flags_from_stat(const float (&v)[KMAX], int kpt, int n, double z,
+                                                uint32_t* flags) {
+  __shared__ double dred[3 * kDW];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  Moments mo{0.0, 0.0, 0.0};
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    if (i < kpt && t + i * kDT < n) {
+      const double f = (double)v[i];
+      mo.n += 1.0;
+      const double dl = f - mo.mean;
+      mo.mean += dl / mo.n;
+      mo.m2 += dl * (f - mo.mean);
+    }
+  }
+  const Moments tot = block_moments<kDT>(mo, dred);
+  const double th = tot.mean + sqrt(tot.m2 / (double)n) * z;
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    if (i < kpt) {
+      const int j = t + i * kDT;
+      const bool k = j < n && (double)v[i] > th;
+      const uint32_t bits = __ballot_sync(0xffffffffu, k);
+      const int w = i * kDW + warp;
+      if (lane == 0 && w < (n + 31) / 32) flags[w] = bits;
+    }
+  }
+}
+
+__device__ __forceinline__ void flags_all_d(int n, uint32_t* flags) {
+  const int nw = (n + 31) / 32;
+  for (int w = threadIdx.x; w < nw; w += kDT) {
+    const int rem = n - w * 32;
+    flags[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+  }
+}
+
+// This CTA's rows: the kept channels whose rank (ascending channel order) is congruent
+// to `part` modulo `parts`, in ascending order, into lrow[0..count). The flag words'
+// exclusive prefix counts go to wpre; each listed rank is then found by a binary search
+// over the words and the position of its set bit within the word. Returns the count
+// (capped at cap; WINA_ERR_CAPACITY is recorded if it does not fit).
+__device__ int list_rows(const uint32_t* flags, int n, int parts, int part, uint32_t* wpre, int* lrow, int cap,
+                         int32_t* status) {
+  __shared__ uint32_t red[kDW + 1];
+  __shared__ uint32_t s_total;
+  const int t = threadIdx.x;
+  const int nw = (n + 31) / 32;  // <= kDMaxN / 32 = 512 < kDT: one word per thread
+  const uint32_t f = t < nw ? flags[t] : 0u;
+  uint32_t tot;
+  const uint32_t pre = block_excl_scan<kDT>((uint32_t)__popc(f), red, &tot);
+  if (t < nw) wpre[t] = pre;
+  if (t == 0) s_total = tot;
+  __syncthreads();
+  const uint32_t total = s_total;
+  int cnt = (int)total > part ? (int)((total - (uint32_t)part + (uint32_t)parts - 1u) / (uint32_t)parts) : 0;
+  if (cnt > cap) {
+    if (t == 0) record_status(status, WINA_ERR_CAPACITY);
+    cnt = cap;
+  }
+  for (int i = t; i < cnt; i += kDT) {
+    const uint32_t rank = (uint32_t)part + (uint32_t)i * (uint32_t)parts;
+    int lo = 0, hi = nw - 1;  // the last word whose prefix count is <= rank holds it
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (wpre[mid] <= rank) lo = mid;
+      else hi = mid - 1;
+    }
+    lrow[i] = lo * 32 + (int)__fns(flags[lo], 0u, (int)(rank - wpre[lo]) + 1);
+  }
+  __syncthreads();
+  return cnt;
+}
+
+// ------------------------------------------------------------------------------------
+// streaming the listed rows
+// ------------------------------------------------------------------------------------
+
+// Partial rows of one CTA's product: the two row groups of a CTA whose rows take 512
+// threads store one each; narrower rows (more groups) are summed in SMEM into one.
+__host__ __device__ inline int decode_partials(int V) { return decode_tpr(V) == kDT / 2 ? 2 : 1; }
+
+// This CTA's partial row(s) of sum over the listed rows r of lval[r] * Wt[lrow[r]][0..m),
+// read with 16-byte loads: row p = blockIdx.x * P + q (q < P = decode_partials(V)) of
+// `part` (row stride pstride floats). The CTA is split into NG = kDT / TPR groups of TPR
+// threads; group g takes list entries g, g + NG, ...; thread l of a group owns VPT vectors
+// of each row, those of index l, l + TPR, ... rotated by an offset that differs from CTA
+// to CTA, and keeps U rows in flight. With more than two groups their sums are combined in
+// SMEM (red, at least (NG - 1) * TPR * EPV floats, groups in order) before the store.
+template <bool BF16, int VPT, int U>
+__device__ void stream_rows(const void* __restrict__ Wt, int m, const int* lrow, const float* lval, int cnt,
+                            float* __restrict__ part, int pstride, float* red, uint64_t pol, long long* stamp_loop,
+                            unsigned long long* t_loop) {
+  constexpr int EPV = VecOps<BF16>::EPV;
+  const int V = m / EPV;
+  const int TPR = decode_tpr(V);
+  const int NG = kDT / TPR;
+  const int t = threadIdx.x, g = t / TPR, l = t % TPR;
+  const uint4* base = reinterpret_cast<const uint4*>(Wt);
+  const int rot = (int)(((int64_t)blockIdx.x * V) / gridDim.x);
+  int vid[VPT];  // this thread's vectors of a row (-1: none)
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int v = l + j * TPR;
+    vid[j] = v < V ? (v + rot < V ? v + rot : v + rot - V) : -1;
+  }
+  float acc[VPT][EPV];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) acc[j][e] = 0.f;
+  int r = g;
+  for (; r + (U - 1) * NG < cnt; r += U * NG) {
+    uint4 w[U][VPT];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint4* rp = base + (int64_t)lrow[r + u * NG] * V;
+#pragma unroll
+      for (int j = 0; j < VPT; ++j)
+        if (vid[j] >= 0) w[u][j] = ld_stream_u4(rp + vid[j], pol);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float xv = lval[r + u * NG];
+#pragma unroll
+      for (int j = 0; j < VPT; ++j)
+        if (vid[j] >= 0) VecOps<BF16>::fma(acc[j], w[u][j], xv);
+    }
+  }
+  for (; r < cnt; r += NG) {
+    const uint4* rp = base + (int64_t)lrow[r] * V;
+    const float xv = lval[r];
+#pragma unroll
+    for (int j = 0; j < VPT; ++j)
+      if (vid[j] >= 0) VecOps<BF16>::fma(acc[j], ld_stream_u4(rp + vid[j], pol), xv);
+  }
+  if (t == 0) {
+    if (blockIdx.x == 0) *stamp_loop = clock64();
+    *t_loop = globaltimer_ns();
+  }
+  if (NG == 2) {  // each group stores its own partial row
+    float* out = part + (size_t)(blockIdx.x * 2 + g) * pstride;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      if (vid[j] >= 0) {
+        float4* o = reinterpret_cast<float4*>(out + (int64_t)vid[j] * EPV);
+#pragma unroll
+        for (int q = 0; q < EPV / 4; ++q)
+          __stcg(o + q, make_float4(acc[j][4 * q], acc[j][4 * q + 1], acc[j][4 * q + 2], acc[j][4 * q + 3]));
+      }
+    }
+    return;
+  }
+  float* out = part + (size_t)blockIdx.x * pstride;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    __syncthreads();
+    if (g > 0 && vid[j] >= 0) {
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) red[((g - 1) * TPR + l) * EPV + e] = acc[j][e];
+    }
+    __syncthreads();
+    if (g == 0 && vid[j] >= 0) {
+      for (int gg = 1; gg < NG; ++gg)
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) acc[j][e] += red[((gg - 1) * TPR + l) * EPV + e];
+      float4* o = reinterpret_cast<float4*>(out + (int64_t)vid[j] * EPV);
+#pragma unroll
+      for (int q = 0; q < EPV / 4; ++q)
+        __stcg(o + q, make_float4(acc[j][4 * q], acc[j][4 * q + 1], acc[j][4 * q + 2], acc[j][4 * q + 3]));
+    }
+  }
+  __syncthreads();  // red (which overlays the selection histogram) is free again
+}
+
+// Reduce-scatter of the partial rows: for this CTA's nq (<= 32) float4 columns
+// q0 .. q0 + nq - 1, the sums over rows p in [0, split) and in [split, end) of
+// part[p][4q .. 4q + 3]. Warp w reads rows w, w + 32, ... in turn (lane i column q0 + i, so
+// that each load instruction takes a few whole cache lines of one row); the warps' sums
+// are then added in warp order through SMEM (red: 32 * 32 float4). Fixed order
+// throughout, so the result is bit-reproducible. Thread i < nq receives the column's two
+// sums. Every thread must call it.
+__device__ void reduce_scatter(const float* __restrict__ part, int pstride, int q0, int nq, int split, int end,
+                               float4* red, float4* sa, float4* sb) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane < nq) {
+    const float4* col = reinterpret_cast<const float4*>(part) + q0 + lane;
+    const int rs = pstride / 4;
+#pragma unroll 4
+    for (int p = warp; p < end; p += 32) {
+      const float4 v = __ldcg(col + (size_t)p * rs);
+      if (p < split) {  // warp-uniform
+        a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+      } else {
+        c.x += v.x; c.y += v.y; c.z += v.z; c.w += v.w;
+      }
+    }
+  }
+  float4 r2[2] = {a, c};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1 && split >= end) break;  // uniform
+    red[warp * 32 + lane] = r2[h];
+    __syncthreads();
+    if (t < nq) {
+      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int w = 0; w < 32; ++w) {
+        const float4 v = red[w * 32 + t];
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
+      if (h == 0) *sa = s;
+      else *sb = s;
+    }
+    __syncthreads();
+  }
+}
+
+__device__ __forceinline__ void touch_pages_d(const void* p, size_t bytes) {
+  const char* c = reinterpret_cast<const char*>(p);
+  for (size_t o = (size_t)threadIdx.x << 21; o < bytes; o += (size_t)kDT << 21)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(c + o));
+}
+
+// ------------------------------------------------------------------------------------
+// the kernel
+// ------------------------------------------------------------------------------------
+
+// VB / VE: 16-byte vectors per thread of a gate/up row and of a down row; UB / UE: rows in
+// flight per thread; KA / KC: channels per thread of x (d) and of h (ffn), at most.
+template <bool BF16, int VB, int UB, int VE, int UE, int KA, int KC>
+__global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
+  constexpr uint32_t ESZ = BF16 ? 2u : 4u;
+  extern __shared__ __align__(128) unsigned char smraw[];
+  const int d = a.d, ffn = a.ffn;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smraw);
+  float* red = reinterpret_cast<float*>(smraw);  // overlays hist while streaming
+  uint32_t* flags = reinterpret_cast<uint32_t*>(smraw + a.sm_flags);
+  uint32_t* wpre = reinterpret_cast<uint32_t*>(smraw + a.sm_wpre);
+  int* lrow = reinterpret_cast<int*>(smraw + a.sm_lrow);
+  float* lval = reinterpret_cast<float*>(smraw + a.sm_lval);
+  const int G = gridDim.x, b = blockIdx.x, t = threadIdx.x, warp = t >> 5;
+  const uint64_t pol = l2_evict_first_policy();
+  const int npb = decode_partials(ffn * (int)ESZ / 16), npe = decode_partials(d * (int)ESZ / 16);
+  dstamp(a.stamps, 0);
+  clear_hist(hist);  // for the first selection (the loads of x and c are in flight meanwhile)
+
+  // ---------------- A: this CTA's projection, its kept set, its rows ----------------
+  const bool gate = b < a.Gg;
+  const int parts = gate ? a.Gg : G - a.Gg;
+  const int part = gate ? b : b - a.Gg;
+  const void* wt = gate ? a.wt_gate : a.wt_up;
+  const int kpt_a = (d + kDT - 1) / kDT;
+  if (a.mode == WINA_GATE_TOPK) {
+    const float* c = gate ? a.c_gate : a.c_up;
+    uint32_t key[KA];
+#pragma unroll
+    for (int i = 0; i < KA; ++i) {
+      const int j = t + i * kDT;
+      key[i] = 0u;
+      if (i < kpt_a && j < d) key[i] = __float_as_uint(fabsf(load_elem(a.x, a.xdt, j) * __ldg(c + j)));
+    }
+    touch_pages_d(wt, (size_t)d * ffn * ESZ);
+    __syncthreads();  // the histogram is zero
+    dstamp(a.stamps, 1);
+    const Threshold th = radix_select_regs(key, kpt_a, d, gate ? a.k_gate : a.k_up, hist);
+    dstamp(a.stamps, 2);
+    flags_from_keys(key, kpt_a, d, th, flags);
+  } else if (a.mode == WINA_GATE_STAT) {
+    float v[KA];
+#pragma unroll
+    for (int i = 0; i < KA; ++i) {
+      const int j = t + i * kDT;
+      v[i] = (i < kpt_a && j < d) ? load_elem(a.x, a.xdt, j) : 0.f;
+    }
+    touch_pages_d(wt, (size_t)d * ffn * ESZ);
+    flags_from_stat(v, kpt_a, d, a.z, flags);
+  } else {
+    touch_pages_d(wt, (size_t)d * ffn * ESZ);
+    flags_all_d(d, flags);
+  }
+  __syncthreads();
+  int cnt = list_rows(flags, d, parts, part, wpre, lrow, a.list_cap, a.status);
+  for (int r = t; r < cnt; r += kDT) lval[r] = load_elem(a.x, a.xdt, lrow[r]);
+  if (part == parts - 1) {
+    uint8_t* kb = gate ? a.keep_g : a.keep_u;
+    for (int j = t; j < d; j += kDT) kb[j] = (uint8_t)((flags[j >> 5] >> (j & 31)) & 1u);
+  }
+  __syncthreads();
+  dstamp(a.stamps, 3);
+  dcta_time(a.cta_t, 0);
+
+  // ---------------- B: stream the gate / up rows into this CTA's partial row ----------------
+  stream_rows<BF16, VB, UB>(wt, ffn, lrow, lval, cnt, a.part, a.pstride, red, pol, a.stamps + 4,
+                            a.cta_t + b * 4 + 1);
+  dstamp(a.stamps, 5);
+  // this CTA's columns of h: float4 columns [qc0, qc0 + nqc); their down-gate norms are
+  // read now and used after the barrier
+  const int qc0 = (int)((int64_t)(ffn / 4) * b / G);
+  const int nqc = (int)((int64_t)(ffn / 4) * (b + 1) / G) - qc0;
+  float4 c4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (t < nqc && a.mode == WINA_GATE_TOPK) c4 = __ldg(reinterpret_cast<const float4*>(a.c_down) + qc0 + t);
+  if (!grid_sync_fixed(a.bar, G, a.status)) return;
+  dstamp(a.stamps, 6);
+
+  // ---------------- C1: this CTA's slice of g and u, h and the down scores ----------------
+  touch_pages_d(a.wt_down, (size_t)d * ffn * ESZ);
+  {
+    float4 g4, u4;
+    reduce_scatter(a.part, a.pstride, qc0, nqc, a.Gg * npb, G * npb, reinterpret_cast<float4*>(red), &g4, &u4);
+    if (t < nqc) {
+      const int q = qc0 + t;
+      const float4 h4 = make_float4(silu_d(g4.x) * u4.x, silu_d(g4.y) * u4.y, silu_d(g4.z) * u4.z,
+                                    silu_d(g4.w) * u4.w);
+      __stcg(reinterpret_cast<float4*>(a.h) + q, h4);
+      if (a.mode == WINA_GATE_TOPK)
+        __stcg(reinterpret_cast<uint4*>(a.dkeys) + q,
+               make_uint4(__float_as_uint(fabsf(h4.x * c4.x)), __float_as_uint(fabsf(h4.y * c4.y)),
+                          __float_as_uint(fabsf(h4.z * c4.z)), __float_as_uint(fabsf(h4.w * c4.w))));
+    }
+  }
+  clear_hist(hist);  // for the down selection (red overlays it)
+  dstamp(a.stamps, 7);
+  if (!grid_sync_fixed(a.bar, G, a.status)) return;
+  dstamp(a.stamps, 8);
+
+  // ---------------- C2: the down kept set and this CTA's rows ----------------
+  const int kpt_c = (ffn + kDT - 1) / kDT;
+  if (a.mode == WINA_GATE_TOPK) {
+    uint32_t key[KC];
+#pragma unroll
+    for (int i = 0; i < KC; ++i) {
+      const int j = t + i * kDT;
+      key[i] = (i < kpt_c && j < ffn) ? __ldcg(a.dkeys + j) : 0u;
+    }
+    dstamp(a.stamps, 9);
+    const Threshold th = radix_select_regs(key, kpt_c, ffn, a.k_down, hist);
+    dstamp(a.stamps, 10);
+    flags_from_keys(key, kpt_c, ffn, th, flags);
+  } else if (a.mode == WINA_GATE_STAT) {
+    float hv[KC];
+#pragma unroll
+    for (int i = 0; i < KC; ++i) {
+      const int j = t + i * kDT;
+      hv[i] = (i < kpt_c && j < ffn) ? __ldcg(a.h + j) : 0.f;
+    }
+    flags_from_stat(hv, kpt_c, ffn, a.z, flags);
+  } else {
+    flags_all_d(ffn, flags);
+  }
+  __syncthreads();
+  cnt = list_rows(flags, ffn, G, b, wpre, lrow, a.list_cap, a.status);
+  for (int r = t; r < cnt; r += kDT) lval[r] = __ldcg(a.h + lrow[r]);
+  if (b == G - 1)
+    for (int j = t; j < ffn; j += kDT) a.keep_d[j] = (uint8_t)((flags[j >> 5] >> (j & 31)) & 1u);
+  __syncthreads();
+  dstamp(a.stamps, 11);
+  dcta_time(a.cta_t, 2);
+
+  // ---------------- E: stream the down rows into this CTA's partial row of y ----------------
+  stream_rows<BF16, VE, UE>(a.wt_down, d, lrow, lval, cnt, a.part, a.pstride, red, pol, a.stamps + 12,
+                            a.cta_t + b * 4 + 3);
+  dstamp(a.stamps, 13);
+  if (!grid_sync_fixed(a.bar, G, a.status)) return;
+  dstamp(a.stamps, 14);
+
+  // ---------------- E2: this CTA's slice of y ----------------
+  {
+    const int q0 = (int)((int64_t)(d / 4) * b / G);
+    const int nq = (int)((int64_t)(d / 4) * (b + 1) / G) - q0;
+    float4 y4, unused;
+    reduce_scatter(a.part, a.pstride, q0, nq, G * npe, G * npe, reinterpret_cast<float4*>(red), &y4, &unused);
+    if (t < nq) reinterpret_cast<float4*>(a.y)[q0 + t] = y4;
+  }
+  dstamp(a.stamps, 15);
+}
+
+// rows in flight per thread for a row of VPT vectors per thread (64 registers per thread
+// at 1024 threads)
+template <int VPT>
+struct RowsInFlight {
+  static constexpr int value = VPT == 1 ? 8 : (VPT == 2 ? 4 : (VPT == 3 ? 2 : 1));
+};
+
+template <bool BF16, int VB, int VE, int KA, int KC>
+static void* decode_kernel() {
+  return (void*)k_ffn_decode<BF16, VB, RowsInFlight<VB>::value, VE, RowsInFlight<VE>::value, KA, KC>;
+}
+
+// Instantiations: the decode shapes of the workloads get their own (the row widths and
+// channel counts fixed at compile time, so that the 64 registers of a 1024-thread CTA hold
+// the keys and the rows in flight without spilling); every other shape up to 16384
+// channels and rows of up to 2048 16-byte vectors takes the general one.
+static void* decode_kernel_for(bool bf16, int vb, int ve, int ka, int kc) {
+  if (bf16) {
+    if (vb == 3 && ve == 1 && ka <= 4 && kc <= 12) return decode_kernel<true, 3, 1, 4, 12>();  // Llama-7B, Gemma-2-2B
+    if (vb == 4 && ve == 1 && ka <= 4 && kc <= 16) return decode_kernel<true, 4, 1, 4, 16>();  // Llama-3-8B
+    return decode_kernel<true, 4, 4, 16, 16>();
+  }
+  return decode_kernel<false, 4, 4, 16, 16>();
+}
+
+// Vectors per thread of a row of m elements (0 if the row is too long for this kernel).
+static int decode_vpt(int64_t m, int esz) {
+  const int64_t V = m * esz / 16;
+  const int tpr = decode_tpr((int)std::min<int64_t>(V, 1 << 20));
+  const int64_t vpt = (V + tpr - 1) / tpr;
+  return vpt <= 4 ? (int)vpt : 0;
+}
+
+// Launch the single-token kernel if it takes this shape; returns WINA_ERR_UNSUPPORTED_DTYPE
+// (no launch) when it does not, so that the caller can use the batched path.
+wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int mode, int k_gate, int k_up,
+                                int k_down, double z, float* y, const FfnWs& L, char* w, int32_t* status,
+                                cudaStream_t st) {
+  const bool bf16 = f->wdt == WINA_BF16;
+  const int esz = bf16 ? 2 : 4;
+  const int d = (int)f->d, ffn = (int)f->ffn;
+  if (d > kDMaxN || ffn > kDMaxN) return WINA_ERR_UNSUPPORTED_DTYPE;
+  const int vb = decode_vpt(ffn, esz), ve = decode_vpt(d, esz);
+  if (vb == 0 || ve == 0) return WINA_ERR_UNSUPPORTED_DTYPE;
+  void* kern = decode_kernel_for(bf16, vb, ve, (d + kDT - 1) / kDT, (ffn + kDT - 1) / kDT);
+  if (!kern) return WINA_ERR_UNSUPPORTED_DTYPE;
+  const int sms = device_sm_count();
+  if (sms < 2) return WINA_ERR_CUDA;
+  // gate/up CTA split in proportion to the kept rows (half each when unknown)
+  int G = std::min(sms, kGridCap);
+  int Gg = G / 2;
+  if (mode == WINA_GATE_TOPK && k_gate + k_up > 0) Gg = (int)(((int64_t)G * k_gate + (k_gate + k_up) / 2) / (k_gate + k_up));
+  Gg = std::max(1, std::min(G - 1, Gg));
+  const int nmax = std::max(d, ffn);
+  const int min_parts = std::min(Gg, G - Gg);
+  const int cap = (nmax + min_parts - 1) / min_parts + 1;
+  const int V_b = ffn * esz / 16, V_e = d * esz / 16;
+  const int tb = decode_tpr(V_b), te = decode_tpr(V_e);
+  const int epv = 16 / esz;
+  const int red_floats = std::max((kDT / tb - 1) * tb * epv, (kDT / te - 1) * te * epv);
+  const DecodeSmem SL = decode_smem(nmax, cap, std::max(red_floats, 32 * 32 * 4));
+  const size_t smem = SL.total;
+  // a CTA's slice of the columns must fit one lane each in reduce_scatter
+  if ((ffn / 4 + G - 1) / G > 32 || (d / 4 + G - 1) / G > 32) return WINA_ERR_UNSUPPORTED_DTYPE;
+  if (blocks_per_sm(kern, kDT, smem) < 1) return WINA_ERR_UNSUPPORTED_DTYPE;
+  DecodeParams p;
+  p.wt_gate = f->wt_gate;
+  p.wt_up = f->wt_up;
+  p.wt_down = f->wt_down;
+  p.c_gate = f->c_gate;
+  p.c_up = f->c_up;
+  p.c_down = f->c_down;
+  p.x = x;
+  p.xdt = xdt;
+  p.d = d;
+  p.ffn = ffn;
+  p.mode = mode;
+  p.k_gate = k_gate;
+  p.k_up = k_up;
+  p.k_down = k_down;
+  p.z = z;
+  p.y = y;
+  p.Gg = Gg;
+  p.list_cap = cap;
+  p.sm_flags = SL.flags;
+  p.sm_wpre = SL.wpre;
+  p.sm_lrow = SL.lrow;
+  p.sm_lval = SL.lval;
+  p.bar = reinterpret_cast<GridBarrier*>(w + L.bar);
+  p.part = reinterpret_cast<float*>(w + L.part);
+  p.pstride = (int)L.pstride;
+  p.dkeys = reinterpret_cast<uint32_t*>(w + L.dkeys);
+  p.h = reinterpret_cast<float*>(w + L.h);
+  p.keep_g = reinterpret_cast<uint8_t*>(w + L.keep_g);
+  p.keep_u = reinterpret_cast<uint8_t*>(w + L.keep_u);
+  p.keep_d = reinterpret_cast<uint8_t*>(w + L.keep_d);
+  p.stamps = reinterpret_cast<long long*>(w + L.stamps);
+  p.cta_t = reinterpret_cast<unsigned long long*>(w + L.cta_t);
+  p.status = status;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)G);
+  cfg.blockDim = dim3(kDT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (smem > 48 * 1024) {
+    cudaError_t e = ensure_smem_limit(kern, smem);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  {
+    cudaError_t e = ensure_prefer_l1(kern);  // the weight loads in flight live in L1
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  void* args[] = {&p};
+  return cuda_status(cudaLaunchKernelExC(&cfg, kern, args));
+}
+
+}  // namespace wina

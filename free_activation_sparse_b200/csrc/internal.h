@@ -16,7 +16,7 @@ constexpr int kGridCap = 296;
 constexpr int kNT = 512;          // threads per CTA of the selection / product kernels
 constexpr int kRowChunk = 1024;   // kept rows staged in SMEM at a time by sparse_matvec
 constexpr size_t kAlign = 256;    // alignment of every workspace sub-buffer
-constexpr int kFfnStamps = 16 + 256;  // phase clock stamps + a stage trace the single-token FFN kernel leaves
+constexpr int kFfnStamps = 32;  // phase clock stamps the single-token FFN kernel leaves (16 used)
 
 inline bool valid_dtype(int dt) { return dt == WINA_F32 || dt == WINA_BF16; }
 inline int64_t elem_size(int dt) { return dt == WINA_BF16 ? 2 : 4; }
@@ -34,6 +34,10 @@ int device_sm_count();
 // Raise a kernel's dynamic SMEM limit to at least `smem` bytes on the current device
 // (remembered per device and kernel, so repeated calls cost a table lookup).
 cudaError_t ensure_smem_limit(const void* kern, size_t smem);
+
+// Ask for the smallest shared-memory carveout (the rest of the SM's unified L1/SMEM stays
+// L1) for `kern` on the current device (remembered per device and kernel).
+cudaError_t ensure_prefer_l1(const void* kern);
 
 // Co-resident CTAs per SM of `kern` at this block size and SMEM on the current device
 // (cached per device, kernel, block size and SMEM). 0 on error.
@@ -89,15 +93,14 @@ inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
 }
 
 // sparse_ffn_swiglu (d, ffn, batch):
-//   bar | ctr [8] (three unit counters, -, epoch) | h [B][ffn] | keep_g [B][d] | keep_u [B][d] (bytes)
-//   | keep_d [B][ffn] (bytes) | stamps [kFfnStamps] | cta_t [kGridCap][4]
+//   bar | h [B][ffn] | keep_g [B][d] | keep_u [B][d] | keep_d [B][ffn] (bytes)
+//   | stamps [kFfnStamps] | cta_t [kGridCap][4]
+//   | part [2 * kGridCap][pstride] | dkeys [ffn]        (one token: the single-token kernel)
 //   | idx_gate, idx_up [B][d] | idx_down [B][ffn] | cnt [3][B] | xs_gate, xs_up [B][d]
-//   | xs_down [B][ffn] | g, u [B][ffn]                       (several tokens)
-//   | acc_g, acc_u [2][ffn]                                 (one token)
-//   | spmv ws                                                 (several tokens)
+//   | xs_down [B][ffn] | g, u [B][ffn] | spmv ws         (the batched path)
 struct FfnWs {
-  size_t bar, ctr, h, keep_g, keep_u, keep_d, stamps, cta_t, idx_gate, idx_up, idx_down, cnt, xs_gate,
-      xs_up, xs_down, g, u, acc_g, acc_u, spmv, total;
+  size_t bar, h, keep_g, keep_u, keep_d, stamps, cta_t, part, pstride, dkeys, idx_gate, idx_up, idx_down, cnt,
+      xs_gate, xs_up, xs_down, g, u, spmv, total;
 };
 inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   FfnWs w;
@@ -109,26 +112,30 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   };
   const bool one = B == 1;
   w.bar = take(sizeof(GridBarrier));
-  w.ctr = take(32);
   w.h = take((size_t)B * ffn * 4);
   w.keep_g = take((size_t)B * d);
   w.keep_u = take((size_t)B * d);
   w.keep_d = take((size_t)B * ffn);
   w.stamps = take((size_t)kFfnStamps * 8);
   w.cta_t = take((size_t)kGridCap * 4 * 8);
-  w.idx_gate = take(one ? 0 : (size_t)B * d * 4);
-  w.idx_up = take(one ? 0 : (size_t)B * d * 4);
-  w.idx_down = take(one ? 0 : (size_t)B * ffn * 4);
-  w.cnt = take(one ? 0 : (size_t)3 * B * 4);
-  w.xs_gate = take(one ? 0 : (size_t)B * d * 4);
-  w.xs_up = take(one ? 0 : (size_t)B * d * 4);
-  w.xs_down = take(one ? 0 : (size_t)B * ffn * 4);
-  w.g = take(one ? 0 : (size_t)B * ffn * 4);
-  w.u = take(one ? 0 : (size_t)B * ffn * 4);
-  w.acc_g = take(one ? (size_t)2 * ffn * 4 : 0);
-  w.acc_u = take(one ? (size_t)2 * ffn * 4 : 0);
+  // partial rows: a multiple of 4 floats plus 4, so that the same column of successive
+  // rows (read together when the rows are summed) does not fall on one L2 slice
+  w.pstride = (size_t)((ffn > d ? ffn : d) + 3) / 4 * 4 + 4;
+  w.part = take(one ? (size_t)2 * kGridCap * w.pstride * 4 : 0);
+  w.dkeys = take(one ? (size_t)ffn * 4 : 0);
+  // the batched path (several tokens, or one token of a shape the single-token kernel
+  // does not take)
+  w.idx_gate = take((size_t)B * d * 4);
+  w.idx_up = take((size_t)B * d * 4);
+  w.idx_down = take((size_t)B * ffn * 4);
+  w.cnt = take((size_t)3 * B * 4);
+  w.xs_gate = take((size_t)B * d * 4);
+  w.xs_up = take((size_t)B * d * 4);
+  w.xs_down = take((size_t)B * ffn * 4);
+  w.g = take((size_t)B * ffn * 4);
+  w.u = take((size_t)B * ffn * 4);
   const int64_t mmax = ffn > d ? ffn : d;
-  w.spmv = take(one ? 0 : spmv_ws_layout(mmax, B).total);
+  w.spmv = take(spmv_ws_layout(mmax, B).total);
   w.total = o;
   return w;
 }
@@ -145,5 +152,10 @@ wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m
                                    const float* xs, int k, const int32_t* count, int ld_idx, int batch, float* y,
                                    void* ws, int32_t* status_dev, cudaStream_t s);
 wina_status_t launch_silu_mul(const float* g, const float* u, float* h, int64_t count, cudaStream_t s);
+// The single-token FFN kernel (ffn_decode.cu). Returns WINA_ERR_UNSUPPORTED_DTYPE without
+// launching anything when the shape is outside what it takes.
+wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int mode, int k_gate, int k_up,
+                                int k_down, double z, float* y, const FfnWs& L, char* w, int32_t* status,
+                                cudaStream_t st);
 
 }  // namespace wina

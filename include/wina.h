@@ -106,15 +106,17 @@ typedef struct {
  *   keep_up   uint8   [batch][d]    1 where the up projection's input channel was kept
  *   keep_down uint8   [batch][ffn]  1 where the down projection's input channel was kept
  *   stamps    int64   [16]          single-token kernel only: SM clock (clock64) of CTA 0
- *                                   at its phase boundaries: 0 start, 10 x and c landed,
- *                                   11 gate/up scores made, 12 boundary bin found,
- *                                   13 channels outside it flagged, 1 gate/up kept sets
- *                                   known, 2 gate/up rows streamed, 3 grid barrier passed,
- *                                   4 h and down scores made, 14 / 15 as 12 / 13 for down,
- *                                   5 down kept set known, 6 its bytes written, 7 down
- *                                   rows streamed, 8 / 9 end
+ *                                   at its phase boundaries: 0 start, 1 gate/up scores
+ *                                   made, 2 kept set found, 3 rows listed, 4 gate/up rows
+ *                                   streamed, 5 partial rows stored, 6 first grid barrier
+ *                                   passed, 7 its slice of h and the down scores written,
+ *                                   8 second barrier passed, 9 down scores loaded, 10 down
+ *                                   kept set found, 11 rows listed, 12 down rows streamed,
+ *                                   13 partial rows stored, 14 third barrier passed,
+ *                                   15 its slice of y written
  *   cta_t     uint64  [CTAs][4]     single-token kernel only: global timer (ns) at which
- *                                   each CTA finished phases 1, 2, 6 and 7 above        */
+ *                                   each CTA finished listing its gate/up rows, streaming
+ *                                   them, listing its down rows and streaming them       */
 typedef struct {
   size_t h;
   size_t keep_gate;
@@ -254,16 +256,20 @@ wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt, int64_t n,
  *   h   = silu(g) * u                (float32; silu(g) = g / (1 + e^-g))
  *   S_d = gate(h, c_down, k_down);  y = W_down[:, S_d] h[S_d]
  * With WINA_GATE_STAT every gate is the Spark threshold with keep fraction s on the
- * projection's signed input (k_* ignored); with WINA_GATE_DENSE every channel is kept.
- * One token (with d, ffn at most 16384 bf16 / 8192 f32 elements) runs as one persistent
- * cooperative kernel: each SM works on the gate or the up projection, selects that
- * projection's kept channels itself, streams its own block of channels' kept weight rows
- * HBM -> SMEM with bulk copies through a ring of stages, then takes units of channels from
- * a global counter; one grid barrier (bounded wait) makes g and u complete; every SM then
- * selects the down projection's kept channels itself and streams its share of those rows,
- * adding into y. Kept sets are exact; y's float32 summation order is not fixed, so repeated
- * calls agree to float32 rounding. Several tokens (or wider shapes) run as a sequence of
- * the batched calls above.
+ * projection's signed input (k_* ignored; gate and up then share one kept set); with
+ * WINA_GATE_DENSE every channel is kept.
+ * One token (d, ffn <= 16384) runs as one persistent cooperative kernel with one CTA of
+ * 1024 threads per SM: each SM works on the gate or the up projection, selects that
+ * projection's kept channels itself (the keys in registers, a radix select on their
+ * bits), takes every (number of SMs on that projection)-th kept row in ascending order
+ * and streams those rows with 16-byte loads into a partial row of g or u; after a grid
+ * barrier each SM sums its slice of the columns over all partial rows in a fixed order
+ * and writes h and the down scores for it; after a second barrier every SM selects the
+ * down kept set and streams its share of those rows into a partial row of y, which a
+ * third barrier and a last fixed-order slice sum turn into y. Every barrier wait is
+ * bounded in time. Kept sets are exact and every sum is taken in a fixed order, so
+ * repeated calls give identical bits. Several tokens (or wider shapes) run as a sequence
+ * of the batched calls above.
  *   f:   host pointer to the weight descriptor (read during the call only).
  *   x:   device [batch][d] of xdt.   y: device float32 [batch][d] (written).
  *   k_gate, k_up in [0, d]; k_down in [0, ffn] (WINA_GATE_TOPK).  0 < s < 1 (STAT).

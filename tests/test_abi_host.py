@@ -53,8 +53,10 @@ def test_workspace_sizes():
     assert s1 >= 296 * 11008 * 4
     assert W.workspace_size(W.OP_SPARSE_MATVEC, 4096, 11008, 2048, 4096) < s1  # one CTA per token: no partials
     f1 = W.workspace_size(W.OP_FFN_SWIGLU, 4096, 11008, 0, 1)
-    assert f1 >= 2 * 2 * 11008 * 4  # double-buffered g/u sums
-    assert W.workspace_size(W.OP_FFN_SWIGLU, 4096, 11008, 0, 4) > f1  # several tokens: per-token buffers
+    assert f1 >= 2 * 296 * 11008 * 4  # the single-token kernel's partial rows (two per CTA)
+    f4 = W.workspace_size(W.OP_FFN_SWIGLU, 4096, 11008, 0, 4)
+    f8 = W.workspace_size(W.OP_FFN_SWIGLU, 4096, 11008, 0, 8)
+    assert f8 > f4 >= 4 * (2 * 4096 + 11008) * 8  # several tokens: per-token index and value lists
     assert W.workspace_size(W.OP_SELECT_TOPK, 10, 10, 1, 1) == 0
     assert W.workspace_size(W.OP_FFN_SWIGLU, 0, 10, 0, 1) == 0
 

@@ -112,9 +112,9 @@ def test_llama7b_dense_mode(llama7b):
 
 
 def test_llama7b_repeatable(llama7b):
-    # The single-token kernel hands out work units dynamically, so the float32 summation
-    # order of the products (not the kept sets of gate and up) can change between calls:
-    # repeated calls must keep the same gate/up sets and agree to float32 rounding.
+    # The single-token kernel sums every product in a fixed order (partial rows reduced
+    # slice by slice, no atomics), so repeated calls give identical bits: the same kept
+    # sets, the same h and the same y.
     cfg, f, *_ = llama7b
     ws = W.Workspace(W.OP_FFN_SWIGLU, 4096, 11008, 0, 1)
     xb = dev_bf16(cfg["x"][:1])
@@ -123,9 +123,9 @@ def test_llama7b_repeatable(llama7b):
     for _ in range(5):
         b = host(W.sparse_ffn_swiglu(f, xb, W.GATE_TOPK, 2048, 2048, 5504, ws=ws))
         v = W.ffn_ws_view(ws, 4096, 11008, 1)
-        assert np.array_equal(host(v["keep_gate"]), v0["keep_gate"])
-        assert np.array_equal(host(v["keep_up"]), v0["keep_up"])
-        assert rel_l2(b, a) <= 1e-5
+        for k in ("keep_gate", "keep_up", "keep_down", "h"):
+            assert np.array_equal(host(v[k]), v0[k]), k
+        assert np.array_equal(b, a)
 
 
 @pytest.mark.parametrize("d,ffn,dt", [(64, 128, "bf16"), (512, 1024, "f32"), (2304, 9216, "bf16"), (8, 16, "f32")])
