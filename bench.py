@@ -272,8 +272,9 @@ def measure_ultrasparse(W, torch, stream, steps: int, copies: int = 2) -> dict:
     ms = _events(torch, stream, step, steps)
     us = ms / (steps * copies) * 1e3
     return {"us_per_call": us, "effective_gbs": nbytes / (us * 1e-6) / 1e9, "union_columns": union,
-            "bytes_per_call": nbytes, "tensor_pipe": "not used (per-token CUDA-core products)",
-            "path": "wina_select_topk (nonzero set) + sparse_matvec, eager calls"}
+            "bytes_per_call": nbytes,
+            "path": "wina_select_topk (nonzero set) + sparse_matvec (union of the 256 tokens' rows, "
+                    "tcgen05 MMA over the gathered union rows), eager calls"}
 
 
 def reduce_max(v: float, world: int, device: str) -> float:
@@ -483,7 +484,7 @@ def main():
     batched = {"batch": BT, "us_per_layer": batched_ms / nb_steps * 1e3 / L,
                "effective_gbs": world * union_bytes * nb_steps / (batched_ms * 1e-3) / 1e9,
                "union_bytes_per_layer": union_bytes // L,
-               "path": "batched calls (select, sparse product, silu*mul) per token group, eager"}
+               "path": "batched calls: select, union-row tcgen05 product, silu*mul (per projection), eager"}
     del xbs, yb, wsb
 
     # end to end through the C ABI: host x in pinned memory -> device, the call, y -> host

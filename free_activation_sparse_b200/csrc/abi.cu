@@ -157,7 +157,7 @@ extern "C" size_t wina_workspace_size(wina_op_t op, int64_t n, int64_t m, int64_
   (void)k;
   if (n < 1 || m < 1 || batch < 1) return 0;
   switch (op) {
-    case WINA_OP_SPARSE_MATVEC: return spmv_ws_layout(m, batch).total;
+    case WINA_OP_SPARSE_MATVEC: return spmv_total_ws(n, m, batch);
     case WINA_OP_FFN_SWIGLU: return ffn_ws_layout(n, m, batch).total;
     default: return 0;
   }

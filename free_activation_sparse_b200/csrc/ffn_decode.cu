@@ -71,7 +71,7 @@ struct DecodeParams {
 };
 
 // Dynamic SMEM: hist [kSelBins + 256] | flags [nw] | word prefix [nw] | list rows [cap] |
-// list values [cap] | group reduction [red_floats] (overlays hist).
+// list values [cap]; the group and slice reductions (red) overlay hist.
 struct DecodeSmem {
   uint32_t hist, flags, wpre, lrow, lval, total;
 };
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   uint32_t* wpre = reinterpret_cast<uint32_t*>(smraw + a.sm_wpre);
   int* lrow = reinterpret_cast<int*>(smraw + a.sm_lrow);
   float* lval = reinterpret_cast<float*>(smraw + a.sm_lval);
-  const int G = gridDim.x, b = blockIdx.x, t = threadIdx.x, warp = t >> 5;
+  const int G = gridDim.x, b = blockIdx.x, t = threadIdx.x;
   const uint64_t pol = l2_evict_first_policy();
   const int npb = decode_partials(ffn * (int)ESZ / 16), npe = decode_partials(d * (int)ESZ / 16);
   dstamp(a.stamps, 0);

@@ -92,6 +92,27 @@ inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
   return w;
 }
 
+// The union path of the sparse product (several tokens, bf16 weights): a byte flag per
+// channel [n], per 64-channel block its first X~ column [nblk], the chunk list [nblk + 1],
+// the channel of each gather slot [kmax], each member's X~ column [n], chunk counts and
+// the number of bf16 parts [4], and X~ [3 * np][kmax] bf16 (np = tokens per block rounded
+// up to 16, kmax = 64 * (nblk + 1)).
+struct UnionWs {
+  size_t flag, base, chunk_row, slot, pos, info, xt, total;
+  int64_t kmax, np;
+};
+UnionWs union_ws_layout(int64_t n, int64_t batch);
+// Whether the union path serves this call (bf16 weights, several tokens).
+bool union_path_takes(int wdt, int64_t n, int64_t m, int64_t batch);
+constexpr int kUnionMinBatch = 4;  // fewer tokens take the per-token product
+
+// sparse_matvec's workspace: the per-token layout, then the union path's (several tokens)
+inline size_t spmv_total_ws(int64_t n, int64_t m, int64_t batch) {
+  size_t t = spmv_ws_layout(m, batch).total;
+  if (batch >= kUnionMinBatch) t += union_ws_layout(n, batch).total;
+  return t;
+}
+
 // sparse_ffn_swiglu (d, ffn, batch):
 //   bar | h [B][ffn] | keep_g [B][d] | keep_u [B][d] | keep_d [B][ffn] (bytes)
 //   | stamps [kFfnStamps] | cta_t [kGridCap][4]
@@ -135,7 +156,7 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   w.g = take((size_t)B * ffn * 4);
   w.u = take((size_t)B * ffn * 4);
   const int64_t mmax = ffn > d ? ffn : d;
-  w.spmv = take(spmv_ws_layout(mmax, B).total);
+  w.spmv = take(spmv_total_ws(mmax, mmax, B));
   w.total = o;
   return w;
 }
@@ -152,6 +173,10 @@ wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m
                                    const float* xs, int k, const int32_t* count, int ld_idx, int batch, float* y,
                                    void* ws, int32_t* status_dev, cudaStream_t s);
 wina_status_t launch_silu_mul(const float* g, const float* u, float* h, int64_t count, cudaStream_t s);
+// The union path (union_gemm.cu); ws is the union region of the workspace.
+wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const int32_t* idx, const float* xs, int k,
+                                  const int32_t* count, int ld, int batch, float* y, void* ws, int32_t* status,
+                                  cudaStream_t s);
 // The single-token FFN kernel (ffn_decode.cu). Returns WINA_ERR_UNSUPPORTED_DTYPE without
 // launching anything when the shape is outside what it takes.
 wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int mode, int k_gate, int k_up,

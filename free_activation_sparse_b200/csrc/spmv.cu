@@ -137,6 +137,9 @@ static size_t spmv_smem() { return (size_t)kRowChunk * 8 + (size_t)kNT * 8 * 4; 
 wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx,
                                    const float* xs, int k, const int32_t* count, int ld_idx, int batch, float* y,
                                    void* ws, int32_t* status_dev, cudaStream_t s) {
+  if (batch >= kUnionMinBatch && union_path_takes(wdt, n, m, batch))
+    return launch_union_matvec(Wt, n, m, idx, xs, k, count, ld_idx, batch, y,
+                               (char*)ws + spmv_ws_layout(m, batch).total, status_dev, s);
   const bool bf16 = wdt == WINA_BF16;
   const size_t smem = spmv_smem();
   const int gmax = bf16 ? max_coresident_grid(k_sparse_matvec<true>, kNT, smem)
