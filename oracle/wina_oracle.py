@@ -52,6 +52,7 @@ __all__ = [
     "silu",
     "ffn_swiglu",
     "spark_threshold",
+    "spark_ffn",
     "exact_topk_signed",
     "overlap",
     "output_error",
@@ -231,6 +232,32 @@ def spark_threshold(v, s: float) -> dict:
     t = mu + sigma * z
     idx = np.nonzero(v > t)[0].astype(np.int32)
     return dict(mu=mu, var=var, sigma=sigma, z=z, t=t, idx=idx)
+
+
+def spark_ffn(Wg, Wu, Wd, x, s: float) -> dict:
+    """The Spark FFN as a key-value lookup ([Spark] section 2.1: y = sum_i f(q . k_i) v_i;
+    compute the dot products of the query with every key, keep the neurons the
+    statistical top-k selects, activate only those), for a SwiGLU FFN:
+
+      g   = W_gate x                         (every neuron's pre-activation: the scores)
+      S   = spark_threshold(g, s)             ([Spark] section 2.2, on the signed float32 g)
+      h_i = silu(g_i) * (W_up[i] . x)   for i in S
+      y   = W_down[:, S] h[S]
+
+    Weights are [out][in]: W_gate, W_up [ffn][d], W_down [d][ffn]. float64 arithmetic; g
+    is held in float32 for the selection (as the scores of the gate are).
+    """
+    Wg = np.asarray(Wg, dtype=np.float64)
+    Wu = np.asarray(Wu, dtype=np.float64)
+    Wd = np.asarray(Wd, dtype=np.float64)
+    x64 = np.asarray(x, dtype=np.float64)
+    g = Wg @ x64
+    g32 = g.astype(np.float32)
+    S = spark_threshold(g32, s)["idx"]
+    u = Wu[S] @ x64
+    h = silu(g[S]) * u
+    y = Wd[:, S] @ h if S.size else np.zeros(Wd.shape[0])
+    return dict(g=g, g32=g32, idx=S, u=u, h=h, y=y)
 
 
 def exact_topk_signed(v, k: int) -> np.ndarray:

@@ -107,6 +107,28 @@ def _ffn_stat_variant(abs_x=False, up_from_xc=False, h64=False):
     return ffn
 
 
+def _spark_ffn_abs_scores(Wg, Wu, Wd, x, s):
+    # thresholds |g| instead of the signed scores
+    Wg = np.asarray(Wg, dtype=np.float64)
+    x64 = np.asarray(x, dtype=np.float64)
+    g = Wg @ x64
+    S = W.spark_threshold(np.abs(g).astype(np.float32), s)["idx"]
+    u = np.asarray(Wu, dtype=np.float64)[S] @ x64
+    h = W.silu(g[S]) * u
+    return dict(g=g, g32=g.astype(np.float32), idx=S, u=u, h=h, y=np.asarray(Wd, dtype=np.float64)[:, S] @ h)
+
+
+def _spark_ffn_swapped_gate(Wg, Wu, Wd, x, s):
+    # silu on the up projection instead of the gate
+    Wg = np.asarray(Wg, dtype=np.float64)
+    x64 = np.asarray(x, dtype=np.float64)
+    g = Wg @ x64
+    S = W.spark_threshold(g.astype(np.float32), s)["idx"]
+    u = np.asarray(Wu, dtype=np.float64)[S] @ x64
+    h = W.silu(u) * g[S]
+    return dict(g=g, g32=g.astype(np.float32), idx=S, u=u, h=h, y=np.asarray(Wd, dtype=np.float64)[:, S] @ h)
+
+
 def _svd_transposed(Wm):
     # transposed operand: W V^T instead of W V
     W64 = np.asarray(Wm, dtype=np.float64)
@@ -128,6 +150,8 @@ MUTATIONS = {
     "ffn_swiglu:stat-gate-on-abs-x": ("ffn_swiglu", _ffn_stat_variant(abs_x=True)),
     "ffn_swiglu:stat-up-set-from-x-times-c": ("ffn_swiglu", _ffn_stat_variant(up_from_xc=True)),
     "ffn_swiglu:stat-down-gate-on-float64-h": ("ffn_swiglu", _ffn_stat_variant(h64=True)),
+    "spark_ffn:abs-scores": ("spark_ffn", _spark_ffn_abs_scores),
+    "spark_ffn:silu-on-up": ("spark_ffn", _spark_ffn_swapped_gate),
 }
 
 PINS = [
@@ -140,6 +164,7 @@ PINS = [
     P.test_silu_closed_forms,
     P.test_ffn_identity_weights_hand_computed,
     P.test_golden_spark_ffn_example,
+    P.test_golden_spark_ffn_lookup,
     P.test_gate_scores_single_fp32_multiply,
     lambda: P.test_spark_keep_fraction_gaussian(2304, 2e-3, 0.03),
     P.test_svd_transform_orthogonal_columns_and_norms,

@@ -434,6 +434,26 @@ def test_golden_spark_ffn_example():
     assert r["y"].tolist() == g["y"]
 
 
+def test_golden_spark_ffn_lookup():
+    # Spark FFN as a key-value lookup: dense scores, statistical top-k on them, only the
+    # selected neurons' up rows and down columns used
+    g = _read_golden("spark_ffn_lookup_worked_example.txt")
+    x = np.array(g["x"])
+    Wg = np.array([g[f"Wg_row{i}"] for i in range(5)])
+    Wu = np.full((5, 3), 9.0)
+    Wu[3], Wu[4] = g["Wu_row3"], g["Wu_row4"]
+    Wd = np.full((3, 5), 5.0)
+    Wd[:, 3], Wd[:, 4] = g["Wd_col3"], g["Wd_col4"]
+    s = 0.5 * math.erfc(g["z"][0] / math.sqrt(2.0))  # 1 - Phi(z)
+    r = O.spark_ffn(Wg, Wu, Wd, x, s)
+    assert r["g"].tolist() == [-2.0, 0.0, 1.0, 4.0, 7.0]
+    assert r["idx"].tolist() == [int(v) for v in g["keep"]]
+    h3 = 16.0 / (1.0 + math.exp(-4.0))
+    h4 = 7.0 / (1.0 + math.exp(-7.0))
+    assert np.allclose(r["h"], [h3, h4], rtol=1e-15, atol=0)
+    assert np.allclose(r["y"], [h3, h4, 2 * h3 + h4], rtol=1e-15, atol=0)
+
+
 def test_ffn_gate_and_up_use_their_own_norms():
     # gate and up see the same x but different c: their kept sets must differ
     x = np.array([1.0, 1.0, 1.0, 1.0], dtype=np.float32)
