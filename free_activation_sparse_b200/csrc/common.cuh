@@ -507,8 +507,10 @@ __device__ __forceinline__ bool grid_sync(GridBarrier* bar, unsigned nblocks, in
 // Barrier for kernels whose grid size never changes for a given workspace: arrivals
 // accumulate in a 64-bit counter, so barrier k of the workspace's life completes when
 // the counter reaches (k + 1) * nblocks. One release atomic per CTA and acquire polls;
-// the last arriver does no extra round trip. Same failure contract as grid_sync.
-__device__ __forceinline__ bool grid_sync_fixed(GridBarrier* bar, unsigned nblocks, int32_t* status) {
+// the last arriver does no extra round trip. Same failure contract as grid_sync, with
+// the wait limit given by the caller.
+__device__ __forceinline__ bool grid_sync_fixed(GridBarrier* bar, unsigned nblocks, int32_t* status,
+                                                unsigned long long limit_ns = kBarrierTimeoutNs) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -518,7 +520,7 @@ __device__ __forceinline__ bool grid_sync_fixed(GridBarrier* bar, unsigned nbloc
     if (ld_acquire_u64(&bar->total) < target) {
       const unsigned long long t0 = globaltimer_ns();
       while (ld_acquire_u64(&bar->total) < target) {
-        if (globaltimer_ns() - t0 > kBarrierTimeoutNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
           ok = 0;
           record_status(status, WINA_ERR_TIMEOUT);
           break;

@@ -2,15 +2,18 @@
 //
 //  * wina_select_topk ("WINA" article, section 一): score_i = |x_i * c_i| in float32,
 //    keep the K largest (ties to the lower index), written as an ascending index list.
-//    One CTA per token: scores live in SMEM as uint32 bit patterns, a histogram select
-//    finds the K-th largest as a threshold, a two-walk warp-ballot compaction emits the
-//    kept indices in ascending order.
+//    Vectors of up to 16384 channels: one CTA of 1024 threads per token keeps the scores'
+//    bit patterns in registers and finds the kept set by a radix select on them; longer
+//    vectors: one CTA per token with the scores in SMEM, a histogram select finds the
+//    K-th largest as a threshold, a two-walk warp-ballot compaction emits the kept
+//    indices in ascending order.
 //  * stat_topk_threshold ("Spark Transformer", section 2.2): mu, sigma^2 (divisor n) in
 //    one pass (Welford per thread, Chan's merge across threads, float64), then
 //    t = mu + sigma * z with z = Phi^-1(1 - s) from the host, keep {i : v_i > t}.
 #include <math.h>
 
 #include "internal.h"
+#include "regsel.cuh"
 
 namespace wina {
 
@@ -45,6 +48,49 @@ __global__ void __launch_bounds__(NT) k_select_topk(const void* __restrict__ x, 
         idx[ob + pos] = i;
         if (xs) xs[ob + pos] = load_elem(x, xdt, off + i);
       });
+}
+
+// The same gate for vectors of up to 16384 channels: one CTA of 1024 threads per token with
+// the keys in registers (radix select on their bits), then the kept channels' flags, a
+// block scan of the flag words' counts and each word's kept channels written in order.
+template <int KMAX>
+__global__ void __launch_bounds__(kDT, 1) k_select_topk_regs(const void* __restrict__ x, int xdt,
+                                                             const float* __restrict__ c, int n, int K, int ld,
+                                                             int32_t* __restrict__ idx, float* __restrict__ xs,
+                                                             float* __restrict__ scores) {
+  __shared__ uint32_t hist[kSelBins + 256];
+  __shared__ uint32_t flags[kDMaxN / 32];
+  __shared__ uint32_t red[kDW + 1];
+  const int t = threadIdx.x;
+  const int64_t off = (int64_t)blockIdx.x * n;
+  const int kpt = (n + kDT - 1) / kDT;
+  clear_hist(hist);
+  uint32_t key[KMAX];
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    const int j = t + i * kDT;
+    key[i] = 0u;
+    if (i < kpt && j < n) {
+      const float xv = load_elem(x, xdt, off + j);
+      const float sv = c ? fabsf(xv * __ldg(c + j)) : fabsf(xv);
+      key[i] = __float_as_uint(sv);
+      if (scores) scores[off + j] = sv;
+    }
+  }
+  __syncthreads();  // the histogram is zero
+  const Threshold th = radix_select_regs(key, kpt, n, K, hist);
+  flags_from_keys(key, kpt, n, th, flags);
+  __syncthreads();
+  const int nw = (n + 31) / 32;  // <= 512 < kDT: one word per thread
+  const uint32_t f = t < nw ? flags[t] : 0u;
+  uint32_t at = block_excl_scan<kDT>((uint32_t)__popc(f), red, nullptr);
+  const int64_t ob = (int64_t)blockIdx.x * ld;
+  for (uint32_t bits = f; bits; bits &= bits - 1u) {
+    const int j = t * 32 + __ffs(bits) - 1;
+    idx[ob + at] = j;
+    if (xs) xs[ob + at] = load_elem(x, xdt, off + j);
+    ++at;
+  }
 }
 
 template <int NT>
@@ -91,6 +137,14 @@ __global__ void __launch_bounds__(NT) k_stat_threshold(const void* __restrict__ 
 
 wina_status_t launch_select_topk(const void* x, int xdt, const float* c, int n, int k, int batch, int32_t* idx,
                                  float* xs, int ld, float* scores, cudaStream_t s) {
+  if (n <= kDMaxN) {
+    const int kpt = (n + kDT - 1) / kDT;
+    void (*kern)(const void*, int, const float*, int, int, int, int32_t*, float*, float*) =
+        kpt <= 4 ? k_select_topk_regs<4> : kpt <= 8 ? k_select_topk_regs<8> : kpt <= 12 ? k_select_topk_regs<12>
+                                                                                     : k_select_topk_regs<16>;
+    kern<<<batch, kDT, 0, s>>>(x, xdt, c, n, k, ld, idx, xs, scores);
+    return cuda_status(cudaGetLastError());
+  }
   const size_t smem = (size_t)(n + kSelBins + 2 * kSelCand) * 4;
   return cuda_status(launch_kernel(k_select_topk<kNT>, dim3(batch), dim3(kNT), smem, s, false, x, xdt, c, n, k, ld,
                                    idx, xs, scores));
