@@ -19,6 +19,7 @@ __all__ = [
     "abi_version", "normal_quantile", "workspace_size", "Workspace", "FfnWeights",
     "pack_in_major", "col_norms", "select_topk", "stat_topk_threshold", "sparse_matvec",
     "sparse_ffn_swiglu", "ffn_ws_view", "ffn_prepare", "declared_symbols", "sparse_matvec_noalloc",
+    "dense_matvec", "dense_ffn_swiglu", "spark_ffn",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwina.so")
@@ -29,7 +30,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_DTYPE, ERR_WORKSPACE, ERR_CAPACITY, ERR_CUD
 F32, BF16 = 0, 1
 LAYOUT_OUT_IN, LAYOUT_IN_MAJOR = 0, 1
 GATE_TOPK, GATE_STAT, GATE_DENSE = 0, 1, 2
-OP_SELECT_TOPK, OP_STAT_THRESHOLD, OP_SPARSE_MATVEC, OP_FFN_SWIGLU = 0, 1, 2, 3
+OP_SELECT_TOPK, OP_STAT_THRESHOLD, OP_SPARSE_MATVEC, OP_FFN_SWIGLU, OP_SPARK_FFN = 0, 1, 2, 3, 4
 
 
 class WinaError(RuntimeError):
@@ -59,6 +60,7 @@ def _load() -> ctypes.CDLL:
     E = ctypes.c_int
     sig = {
         "wina_abi_version": (I32, []),
+        "wina_set_wait_limit_ns": (None, [ctypes.c_uint64]),
         "wina_status_string": (ctypes.c_char_p, [E]),
         "wina_normal_quantile": (D, [D]),
         "wina_workspace_size": (SZ, [E, I64, I64, I64, I64]),
@@ -70,6 +72,9 @@ def _load() -> ctypes.CDLL:
         "sparse_matvec": (E, [P, E, I64, I64, P, P, I64, P, I64, I64, P, P, SZ, P, P]),
         "sparse_matvec_noalloc": (E, [P, E, I64, I64, P, P, I64, P, I64, I64, P, P, P]),
         "sparse_ffn_swiglu": (E, [ctypes.POINTER(_FfnT), P, E, I64, E, I64, I64, I64, D, P, P, SZ, P, P]),
+        "wina_dense_matvec": (E, [P, E, I64, I64, P, E, P, P, P]),
+        "spark_ffn_swiglu": (E, [P, P, P, E, I64, I64, P, E, D, P, P, P, P, P, SZ, P, P]),
+        "wina_dense_ffn_swiglu": (E, [P, P, P, E, I64, I64, P, E, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -321,6 +326,57 @@ def sparse_ffn_swiglu(f: FfnWeights, x, mode: int = GATE_TOPK, k_gate: int = 0, 
                                  int(k_down), float(s), _ptr(y), ws.ptr, ws.nbytes, _ptr(status), _stream()),
            "sparse_ffn_swiglu")
     return y
+
+
+def dense_matvec(W, x, y=None, xbuf=None):
+    """The dense comparator y = W x on the output-major W [m][n] (one token)."""
+    torch = _torch()
+    _cuda(W, "W")
+    _cuda(x, "x")
+    m, n = W.shape
+    if y is None:
+        y = torch.empty(m, dtype=torch.float32, device=W.device)
+    if xbuf is None:
+        xbuf = torch.empty(n, dtype=torch.float32, device=W.device)
+    _check(lib.wina_dense_matvec(_ptr(W), _dt(W), m, n, _ptr(x), _dt(x), _ptr(y), _ptr(xbuf), _stream()),
+           "wina_dense_matvec")
+    return y
+
+
+def dense_ffn_swiglu(W_gate, W_up, W_down, x, y=None, buf=None):
+    """The dense comparator of the FFN on the output-major weights (one token): returns y [d]."""
+    torch = _torch()
+    for t_, nm in ((W_gate, "W_gate"), (W_up, "W_up"), (W_down, "W_down"), (x, "x")):
+        _cuda(t_, nm)
+    ffn, d = W_gate.shape
+    if y is None:
+        y = torch.empty(d, dtype=torch.float32, device=x.device)
+    if buf is None:
+        buf = torch.empty((d + 3) // 4 * 4 + ffn, dtype=torch.float32, device=x.device)
+    _check(lib.wina_dense_ffn_swiglu(_ptr(W_gate), _ptr(W_up), _ptr(W_down), _dt(W_gate), d, ffn, _ptr(x), _dt(x),
+                                     _ptr(y), _ptr(buf), _stream()), "wina_dense_ffn_swiglu")
+    return y
+
+
+def spark_ffn(W_gate, W_up, Wt_down, x, s: float = 0.08, ws: Workspace | None = None, status=None, y=None):
+    """The Spark FFN as a key-value lookup for one token: W_gate, W_up output-major [ffn][d],
+    Wt_down input-major [ffn][d]. Returns (y [d], g [ffn], idx [ffn] (first count valid),
+    count [1])."""
+    torch = _torch()
+    for t_, nm in ((W_gate, "W_gate"), (W_up, "W_up"), (Wt_down, "Wt_down"), (x, "x")):
+        _cuda(t_, nm)
+    ffn, d = W_gate.shape
+    if ws is None:
+        ws = Workspace(OP_SPARK_FFN, d, ffn, 0, 1, device=x.device)
+    if y is None:
+        y = torch.empty(d, dtype=torch.float32, device=x.device)
+    g = torch.empty(ffn, dtype=torch.float32, device=x.device)
+    idx = torch.empty(ffn, dtype=torch.int32, device=x.device)
+    count = torch.empty(1, dtype=torch.int32, device=x.device)
+    _check(lib.spark_ffn_swiglu(_ptr(W_gate), _ptr(W_up), _ptr(Wt_down), _dt(W_gate), d, ffn, _ptr(x), _dt(x),
+                                float(s), _ptr(y), _ptr(g), _ptr(idx), _ptr(count), ws.ptr, ws.nbytes, _ptr(status),
+                                _stream()), "spark_ffn_swiglu")
+    return y, g, idx, count
 
 
 def ffn_ws_view(ws: Workspace, d: int, ffn: int, batch: int) -> dict:

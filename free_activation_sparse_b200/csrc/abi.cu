@@ -2,6 +2,7 @@
 // used by the Spark threshold, workspace sizes and workspace views.
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -105,6 +106,12 @@ int blocks_per_sm(const void* kern, int threads, size_t smem) {
   return per_sm;
 }
 
+namespace {
+std::atomic<unsigned long long> g_wait_ns{kBarrierTimeoutNs};
+}  // namespace
+
+unsigned long long wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
 // Phi(z) = P(Z <= z) for a standard normal Z, via the complementary error function.
 static double normal_cdf(double z) { return 0.5 * erfc(-z / sqrt(2.0)); }
 
@@ -113,6 +120,10 @@ static double normal_cdf(double z) { return 0.5 * erfc(-z / sqrt(2.0)); }
 using namespace wina;
 
 extern "C" int32_t wina_abi_version(void) { return WINA_ABI_VERSION; }
+
+extern "C" void wina_set_wait_limit_ns(uint64_t ns) {
+  g_wait_ns.store(ns ? (unsigned long long)ns : kBarrierTimeoutNs, std::memory_order_relaxed);
+}
 
 extern "C" const char* wina_status_string(wina_status_t s) {
   switch (s) {
@@ -159,6 +170,7 @@ extern "C" size_t wina_workspace_size(wina_op_t op, int64_t n, int64_t m, int64_
   switch (op) {
     case WINA_OP_SPARSE_MATVEC: return spmv_total_ws(n, m, batch);
     case WINA_OP_FFN_SWIGLU: return ffn_ws_layout(n, m, batch).total;
+    case WINA_OP_SPARK_FFN: return batch == 1 ? spark_ws_size(n, m) : 0;
     default: return 0;
   }
 }

@@ -23,6 +23,9 @@ inline int64_t elem_size(int dt) { return dt == WINA_BF16 ? 2 : 4; }
 inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Time limit of the grid-barrier waits of the single-token FFN kernel (wina_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
+
 inline wina_status_t cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return WINA_OK;
   return WINA_ERR_CUDA;
@@ -173,6 +176,8 @@ wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m
                                    const float* xs, int k, const int32_t* count, int ld_idx, int batch, float* y,
                                    void* ws, int32_t* status_dev, cudaStream_t s);
 wina_status_t launch_silu_mul(const float* g, const float* u, float* h, int64_t count, cudaStream_t s);
+// Workspace bytes of spark_ffn_swiglu (spark.cu).
+size_t spark_ws_size(int64_t d, int64_t ffn);
 // The union path (union_gemm.cu); ws is the union region of the workspace.
 wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const int32_t* idx, const float* xs, int k,
                                   const int32_t* count, int ld, int batch, float* y, void* ws, int32_t* status,

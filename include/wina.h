@@ -80,7 +80,8 @@ typedef enum {
   WINA_OP_SELECT_TOPK = 0,
   WINA_OP_STAT_THRESHOLD = 1,
   WINA_OP_SPARSE_MATVEC = 2,
-  WINA_OP_FFN_SWIGLU = 3
+  WINA_OP_FFN_SWIGLU = 3,
+  WINA_OP_SPARK_FFN = 4
 } wina_op_t;
 
 /* The three projections of a SwiGLU FFN, already packed input-major:
@@ -129,6 +130,13 @@ typedef struct {
 /* ABI version of the loaded library (WINA_ABI_VERSION at build time). */
 int32_t wina_abi_version(void);
 
+/* Test and diagnosis hook (host function): the time limit of each grid-barrier wait of
+ * the single-token sparse_ffn_swiglu kernel, for launches made after the call, process-
+ * wide; 0 restores the default of 1 s. A wait that exceeds it records WINA_ERR_TIMEOUT in
+ * the call's status word and the kernel returns (the workspace must then be zero-filled
+ * again before its next use). */
+void wina_set_wait_limit_ns(uint64_t ns);
+
 /* Static description of a status code (host pointer to a constant string). */
 const char* wina_status_string(wina_status_t status);
 
@@ -148,6 +156,7 @@ double wina_normal_quantile(double p);
  *   WINA_OP_SPARSE_MATVEC: n = in-features, m = out-features, k = max kept per token,
  *                          batch = tokens.
  *   WINA_OP_FFN_SWIGLU:    n = d, m = ffn, k ignored, batch = tokens.
+ *   WINA_OP_SPARK_FFN:     n = d, m = ffn, k ignored, batch = 1.
  *   WINA_OP_SELECT_TOPK, WINA_OP_STAT_THRESHOLD: 0.                                  */
 size_t wina_workspace_size(wina_op_t op, int64_t n, int64_t m, int64_t k, int64_t batch);
 
@@ -280,6 +289,44 @@ wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt, int64_t n,
 wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, wina_dtype_t xdt, int64_t batch,
                                 wina_gate_mode_t mode, int64_t k_gate, int64_t k_up, int64_t k_down, double s,
                                 float* y, void* ws, size_t ws_bytes, int32_t* status_dev, wina_stream_t stream);
+
+/* The Spark FFN as a key-value lookup ("Spark Transformer", section 2.1: y = sum_i
+ * f(q . k_i) v_i, with the statistical top-k of section 2.2 choosing the neurons), for a
+ * SwiGLU FFN and one token:
+ *   g   = W_gate x                 (every neuron's score: dense, all of W_gate is read)
+ *   S   = { i : g_i > mu + sigma * Phi^-1(1 - s) }    (mean, population variance of g)
+ *   h_i = silu(g_i) * (W_up[i] . x)           for i in S   (only the selected rows)
+ *   y   = sum over i in S of h_i * W_down[:, i]            (only the selected columns)
+ *   W_gate, W_up: device [ffn][d] OUTPUT-major (row i is neuron i's key / up row);
+ *   Wt_down: device [ffn][d] input-major (wina_pack_in_major of W_down [d][ffn]);
+ *   x: device [d] of xdt;  y: device float32 [d] (written);
+ *   g_out: device float32 [ffn] or NULL: the scores g (float32);
+ *   idx: device int32 [ffn]: the selected neurons ascending (the first *count valid);
+ *   count: device int32 [1]: |S|;  0 < s < 1;
+ *   ws: device scratch of wina_workspace_size(WINA_OP_SPARK_FFN, d, ffn, 0, 1) bytes.
+ *   d % 8 == 0 (bf16) or % 4 (f32); d, ffn <= 32768. */
+wina_status_t spark_ffn_swiglu(const void* W_gate, const void* W_up, const void* Wt_down, wina_dtype_t wdt,
+                               int64_t d, int64_t ffn, const void* x, wina_dtype_t xdt, double s, float* y,
+                               float* g_out, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                               int32_t* status_dev, wina_stream_t stream);
+
+/* The dense comparator: the unsparsified layer y = W x (every channel kept), on the
+ * OUTPUT-major weight W[m][n] (the matrix that multiplies x, unpacked), one warp per output
+ * row with 16-byte streaming loads; no workspace beyond xbuf. Batch 1.
+ *   W:    device [m][n] of wdt (n % 8 == 0 for bf16, % 4 for f32).
+ *   x:    device [n] of xdt.   y: device float32 [m] (written).
+ *   xbuf: device float32 [n] scratch (x widened), 16-byte aligned. */
+wina_status_t wina_dense_matvec(const void* W, wina_dtype_t wdt, int64_t m, int64_t n, const void* x,
+                                wina_dtype_t xdt, float* y, float* xbuf, wina_stream_t stream);
+
+/* The dense comparator of sparse_ffn_swiglu: y = W_down (silu(W_gate x) * (W_up x)) with
+ * every channel kept, on the output-major weights W_gate, W_up [ffn][d] and W_down
+ * [d][ffn]. Two launches: gate and up rows together (h), then down. Batch 1.
+ *   x: device [d] of xdt;  y: device float32 [d] (written);
+ *   buf: device float32 scratch of round_up(d, 4) + ffn floats, 16-byte aligned. */
+wina_status_t wina_dense_ffn_swiglu(const void* W_gate, const void* W_up, const void* W_down, wina_dtype_t wdt,
+                                    int64_t d, int64_t ffn, const void* x, wina_dtype_t xdt, float* y, float* buf,
+                                    wina_stream_t stream);
 
 #ifdef __cplusplus
 }
