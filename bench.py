@@ -203,78 +203,180 @@ def _events(torch, stream, fn, steps: int) -> float:
     return e0.elapsed_time(e1)
 
 
-def measure_spark_ffn(W, torch, stream, steps: int, copies: int = 4) -> dict:
+def graph_us(torch, fn, steps: int, warm: int = 3) -> float:
+    """Microseconds per call of fn(), captured once as a CUDA graph and replayed `steps`
+    times between two events on the current stream (synchronised on both sides)."""
+    stream = torch.cuda.current_stream()
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        fn()  # warm the library's per-device caches outside capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            fn()
+    torch.cuda.synchronize()
+    for _ in range(warm):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del g
+    return ms * 1e3 / steps
+
+
+def _dev_bf16(torch, bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _frac(nbytes: float, us: float, peak: float) -> dict:
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"us": us, "effective_gbs": gbs, "frac_of_measured_hbm": gbs / peak, "bytes": int(nbytes)}
+
+
+def measure_spark(W, torch, steps: int, peak: float, batches=(1, 2, 4, 8, 16, 32, 64), copies: int = 4) -> dict:
     """Gemma-2-2B FFN (d 2304, ffn 9216, bf16) with the Spark statistical gate (keep
-    fraction 0.08) on every projection, one token per call, `copies` distinct weight
-    copies (4 x 127 MB, above L2) called in turn. Bytes: the kept rows (read back from
-    the call's kept-set views) plus the vectors."""
-    cfg = synth.make_gemma2_2b_spark(batch=1)
+    fraction 0.08) on every projection, `copies` distinct weight copies (4 x 127 MB, above
+    L2) called in turn, for several token counts; and, on the stand-alone Gaussian vectors
+    of the workload (2304 and 9216 long, 64 tokens), the overlap of the Spark set with the
+    exact top-k of the signed values (k = round(s n)), from the GPU's kept sets and a numpy
+    sort. Bytes: the kept rows (read back from the call's kept-set views; the union over
+    the tokens when several) plus the vectors."""
+    cfg = synth.make_gemma2_2b_spark(batch=max(batches))
     d, ffn, s = cfg["d"], cfg["ffn"], cfg["s"]
     fs = []
     for _ in range(copies):
-        up = [torch.from_numpy(cfg[k].view(np.int16)).cuda().view(torch.bfloat16) for k in ("Wg", "Wu", "Wd")]
-        fs.append(W.ffn_prepare(*up))
-        del up
-    x = torch.from_numpy(cfg["x_bf16"].view(np.int16)).cuda().view(torch.bfloat16)
-    ws = W.Workspace(W.OP_FFN_SWIGLU, d, ffn, 0, 1)
-    y = torch.empty((1, d), dtype=torch.float32, device="cuda")
+        fs.append(W.ffn_prepare(*(_dev_bf16(torch, cfg[k]) for k in ("Wg", "Wu", "Wd"))))
+    xall = _dev_bf16(torch, cfg["x_bf16"])
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = {"gate": "Spark statistical top-k, s = 0.08, every projection", "by_batch": {}}
+    for B in batches:
+        x = xall[:B].contiguous()
+        ws = W.Workspace(W.OP_FFN_SWIGLU, d, ffn, 0, B)
+        y = torch.empty((B, d), dtype=torch.float32, device="cuda")
 
-    def step():
-        for f in fs:
-            W.sparse_ffn_swiglu(f, x, W.GATE_STAT, s=s, ws=ws, status=st, y=y)
+        def step():
+            for f in fs:
+                W.sparse_ffn_swiglu(f, x, W.GATE_STAT, s=s, ws=ws, status=st, y=y)
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
-    if int(st.item()) != 0:
-        raise RuntimeError(f"device status {int(st.item())}")
-    v = W.ffn_ws_view(ws, d, ffn, 1)
-    kg, ku, kd = (int(v[k].sum().item()) for k in ("keep_gate", "keep_up", "keep_down"))
-    nbytes = (kg + ku) * ffn * 2 + kd * d * 2 + d * 2 + d * 4
-    ms = _events(torch, stream, step, steps)
-    us = ms / (steps * copies) * 1e3
-    return {"us_per_layer": us, "effective_gbs": nbytes / (us * 1e-6) / 1e9, "bytes_per_layer": nbytes,
-            "kept": [kg, ku, kd], "gate": "Spark statistical top-k, s = 0.08", "path": "fused kernel, eager calls"}
+        us = graph_us(torch, step, steps) / copies
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status {int(st.item())}")
+        v = W.ffn_ws_view(ws, d, ffn, B)
+        kg, ku, kd = (int(v[k].bool().any(0).sum().item()) for k in ("keep_gate", "keep_up", "keep_down"))
+        nbytes = (kg + ku) * ffn * 2 + kd * d * 2 + B * (d * 2 + d * 4)
+        out["by_batch"][str(B)] = dict(_frac(nbytes, us, peak), us_per_layer=us, union_kept=[kg, ku, kd])
+        del ws, y
+    # overlap with the exact top-k of the signed values
+    ov = {}
+    for name, arr in (("x_2304", cfg["x"]), ("v_9216", cfg["v"])):
+        n = arr.shape[1]
+        k = synth.spark_keep_count(s, n)
+        idx, _, cnt, _ = W.stat_topk_threshold(torch.from_numpy(arr).cuda(), s)
+        idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+        rec, jac = [], []
+        for b in range(arr.shape[0]):
+            S = set(idx[b, :cnt[b]].tolist())
+            T = set(np.argsort(-arr[b], kind="stable")[:k].tolist())
+            inter = len(S & T)
+            rec.append(inter / k)
+            jac.append(inter / max(1, len(S | T)))
+        ov[name] = {"k": k, "mean_kept": float(cnt.mean()), "recall_vs_exact_topk": float(np.mean(rec)),
+                    "jaccard": float(np.mean(jac)), "tokens": int(arr.shape[0])}
+    out["overlap_with_exact_topk"] = ov
+    return out
 
 
-def measure_ultrasparse(W, torch, stream, steps: int, copies: int = 2) -> dict:
+def measure_ultrasparse(W, torch, steps: int, peak: float, copies: int = 2) -> dict:
     """Down projection 14336 -> 4096 (bf16), 256 tokens with 143 nonzero inputs each: the
-    nonzero set selected on the GPU and the sparse product, per step; `copies` distinct
-    weight copies (2 x 117 MB) called in turn. Bytes: the union of the tokens' columns
-    (read once by a union product) plus the inputs and outputs."""
+    nonzero set selected on the GPU and the union-row tensor-core product, per step;
+    `copies` distinct weight copies (2 x 117 MB) called in turn, as a CUDA graph. Bytes:
+    the union of the tokens' columns (read once) plus the inputs and outputs."""
     cfg = synth.make_ultrasparse_down()
     n, m, nnz = cfg["n"], cfg["m"], cfg["nnz"]
-    Wts = []
-    for _ in range(copies):
-        Wd = torch.from_numpy(cfg["W"].view(np.int16)).cuda().view(torch.bfloat16)
-        Wts.append(W.pack_in_major(Wd))
-        del Wd
-    xb = torch.from_numpy(cfg["x"].view(np.int16)).cuda().view(torch.bfloat16)
+    Wts = [W.pack_in_major(_dev_bf16(torch, cfg["W"])) for _ in range(copies)]
+    xb = _dev_bf16(torch, cfg["x"])
     B = xb.shape[0]
     ws = W.Workspace(W.OP_SPARSE_MATVEC, n, m, nnz, B)
     y = torch.empty((B, m), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx = torch.empty((B, nnz), dtype=torch.int32, device="cuda")
+    xs = torch.empty((B, nnz), dtype=torch.float32, device="cuda")
 
     def step():
         for Wt in Wts:
-            idx, xs = W.select_topk(xb, None, nnz)
+            W.lib.wina_select_topk(W._ptr(xb), W.BF16, None, n, nnz, B, W._ptr(idx), W._ptr(xs), None, W._stream())
             W.sparse_matvec(Wt, idx, xs, ws=ws, status=st, y=y)
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
+    us = graph_us(torch, step, steps) / copies
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())}")
-    idx, _ = W.select_topk(xb, None, nnz)
     union = int(torch.unique(idx).numel())
     nbytes = union * m * 2 + B * n * 2 + B * m * 4
-    ms = _events(torch, stream, step, steps)
-    us = ms / (steps * copies) * 1e3
-    return {"us_per_call": us, "effective_gbs": nbytes / (us * 1e-6) / 1e9, "union_columns": union,
-            "bytes_per_call": nbytes,
-            "path": "wina_select_topk (nonzero set) + sparse_matvec (union of the 256 tokens' rows, "
-                    "tcgen05 MMA over the gathered union rows), eager calls"}
+    mm = graph_us(torch, lambda: [W.sparse_matvec(Wt, idx, xs, ws=ws, status=st, y=y) for Wt in Wts], steps) / copies
+    return dict(_frac(nbytes, us, peak), us_per_call=us, union_columns=union, product_only_us=mm,
+                useful_gflop=2.0 * m * nnz * B / 1e9, union_mma_gflop=2.0 * m * union * B / 1e9,
+                path="wina_select_topk (nonzero set) + sparse_matvec (union of the 256 tokens' rows on tcgen05)")
+
+
+def measure_llama3_layer(W, torch, steps: int, peak: float, batches=(1, 4, 16)) -> dict:
+    """Llama-3-8B-shaped decoder layer (bf16): Q/K/V/O as gated sparse products (each its
+    own top-K of |input * c|; Q, K, V gate the hidden state, O an independent input since
+    no attention core is in scope) and the gated SwiGLU FFN (gate/up 4096 -> 14336, down
+    14336 -> 4096), per-projection sparsity from the workload's seeded schedule, one layer
+    (436 MB of weights, above L2) per step, as a CUDA graph. Bytes: each projection's kept
+    rows (their union over the tokens) plus the vectors."""
+    cfg = synth.make_llama3_8b_layer(batch=max(batches))
+    k = cfg["k"]
+    Wt, c = {}, {}
+    for name in ("q", "k", "v", "o"):
+        Wd = _dev_bf16(torch, cfg["W"][name])
+        Wt[name], c[name] = W.pack_in_major(Wd), W.col_norms(Wd)
+        del Wd
+    f = W.ffn_prepare(*(_dev_bf16(torch, cfg["W"][nm]) for nm in ("gate", "up", "down")))
+    del cfg["W"]
+    xall = _dev_bf16(torch, cfg["x"])
+    oall = _dev_bf16(torch, cfg["o_in"])
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = {"k": k, "p": cfg["p"], "by_batch": {}}
+    for B in batches:
+        x, o_in = xall[:B].contiguous(), oall[:B].contiguous()
+        sel = {nm: (torch.empty((B, k[nm]), dtype=torch.int32, device="cuda"),
+                    torch.empty((B, k[nm]), dtype=torch.float32, device="cuda")) for nm in ("q", "k", "v", "o")}
+        ys = {nm: torch.empty((B, Wt[nm].shape[1]), dtype=torch.float32, device="cuda") for nm in ("q", "k", "v", "o")}
+        wss = {nm: W.Workspace(W.OP_SPARSE_MATVEC, 4096, Wt[nm].shape[1], k[nm], B) for nm in ("q", "k", "v", "o")}
+        fws = W.Workspace(W.OP_FFN_SWIGLU, 4096, 14336, 0, B)
+        yf = torch.empty((B, 4096), dtype=torch.float32, device="cuda")
+
+        def step():
+            for nm in ("q", "k", "v", "o"):
+                inp = o_in if nm == "o" else x
+                idx, xs = sel[nm]
+                W.lib.wina_select_topk(W._ptr(inp), W.BF16, W._ptr(c[nm]), 4096, k[nm], B, W._ptr(idx), W._ptr(xs),
+                                       None, W._stream())
+                W.sparse_matvec(Wt[nm], idx, xs, ws=wss[nm], status=st, y=ys[nm])
+            W.sparse_ffn_swiglu(f, x, W.GATE_TOPK, k["gate"], k["up"], k["down"], ws=fws, status=st, y=yf)
+
+        us = graph_us(torch, step, steps)
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status {int(st.item())}")
+        nbytes = 0
+        for nm in ("q", "k", "v", "o"):
+            nbytes += int(torch.unique(sel[nm][0]).numel()) * Wt[nm].shape[1] * 2
+        v = W.ffn_ws_view(fws, 4096, 14336, B)
+        ug, uu, ud = (int(v[kk].bool().any(0).sum().item()) for kk in ("keep_gate", "keep_up", "keep_down"))
+        nbytes += (ug + uu) * 14336 * 2 + ud * 4096 * 2 + B * 4096 * 2 * 2
+        out["by_batch"][str(B)] = dict(_frac(nbytes, us, peak), us_per_layer=us,
+                                       path="per-token kernels (B = 1) / union-row tcgen05 products (B >= 4)")
+        del sel, ys, wss, fws, yf
+    return out
 
 
 def reduce_max(v: float, world: int, device: str) -> float:
@@ -349,12 +451,12 @@ def main():
 
     # ---- untimed setup: L layers of weights (packed + norms on the GPU), inputs ----
     L = args.layers
-    layers, xs = [], []
+    layers, xs, outmajor = [], [], []
     for l in range(L):
         cfg = synth.make_llama7b_ffn(batch=1, p=args.p, layer=l + 1000 * rank)
         up = [torch.from_numpy(cfg[k].view(np.int16)).cuda().view(torch.bfloat16) for k in ("Wg", "Wu", "Wd")]
         layers.append(W.ffn_prepare(*up))
-        del up
+        outmajor.append(up)  # the unpacked weights, for the dense comparator
         xs.append(torch.from_numpy(cfg["x"].view(np.int16)).cuda().view(torch.bfloat16))
     torch.cuda.synchronize()
     ws = W.Workspace(W.OP_FFN_SWIGLU, D, FFN, 0, 1)
@@ -437,14 +539,54 @@ def main():
     kern_ms = ms_per_step / L  # graph replay: per-launch time including the gap to the next launch
     gbs = world * nbytes * L * args.steps / (total_ms * 1e-3) / 1e9
 
-    # dense comparator: the same kernel with every channel kept
-    dgraph = capture(W.GATE_DENSE)
-    for _ in range(3):
-        dgraph.replay()
-    nd = max(3, args.steps // 2)
-    dense_ms = max_over_ranks(timed_graph(dgraph, nd))
-    us_layer_dense = dense_ms / nd * 1e3 / L
-    del dgraph
+    peak, peak_kind = _peaks()
+    nsteps = max(3, args.steps // 2)
+
+    # dense comparator: the unsparsified FFN on the output-major weights (dedicated dense
+    # GEMV kernels: one warp per output row, no selection, no cross-CTA sums)
+    dbuf = torch.empty(D + FFN, dtype=torch.float32, device="cuda")
+
+    def dense_step():
+        for l in range(L):
+            W.dense_ffn_swiglu(outmajor[l][0], outmajor[l][1], outmajor[l][2], xs[l][0], y=ys[l][0], buf=dbuf)
+
+    us_layer_dense = max_over_ranks(graph_us(torch, dense_step, nsteps)) / L
+    dense_bytes = 3 * D * FFN * 2 + D * 2 + D * 4
+    # the decode kernel itself with every channel kept (its own dense mode)
+    us_layer_dense_mode = max_over_ranks(graph_us(torch, lambda: step(W.GATE_DENSE), nsteps)) / L
+
+    # the headline layer at 65% sparsity (K = 1434 / 1434 / 3853)
+    kg65, kd65 = synth.keep_count(0.65, D), synth.keep_count(0.65, FFN)
+
+    def step65():
+        for l in range(L):
+            W.sparse_ffn_swiglu(layers[l], xs[l], W.GATE_TOPK, kg65, kg65, kd65, ws=ws, status=status, y=ys[l])
+
+    us65 = max_over_ranks(graph_us(torch, step65, nsteps)) / L
+    p065 = dict(_frac(layer_bytes(kg65, kg65, kd65), us65, peak), us_per_layer=us65, k=[kg65, kg65, kd65])
+
+    # the sparse product alone at batch 1: the gate projection's kept rows (4096 -> 11008,
+    # K = kg) and the down projection's (11008 -> 4096, K = kd, on the h the FFN produced)
+    sel_g, sel_d, yg, ydn = [], [], [], []
+    mws = W.Workspace(W.OP_SPARSE_MATVEC, FFN, FFN, FFN, 1)
+    for l in range(L):
+        sel_g.append(W.select_topk(xs[l], layers[l].c_gate, kg))
+        W.sparse_ffn_swiglu(layers[l], xs[l], W.GATE_TOPK, kg, kg, kd, ws=ws, status=status, y=ys[l])
+        h = W.ffn_ws_view(ws, D, FFN, 1)["h"].clone()
+        sel_d.append(W.select_topk(h, layers[l].c_down, kd))
+        yg.append(torch.empty((1, FFN), dtype=torch.float32, device="cuda"))
+        ydn.append(torch.empty((1, D), dtype=torch.float32, device="cuda"))
+    us_mg = max_over_ranks(graph_us(torch, lambda: [W.sparse_matvec(layers[l].wt_gate, *sel_g[l], ws=mws,
+                                                                    status=status, y=yg[l]) for l in range(L)],
+                                    nsteps)) / L
+    us_md = max_over_ranks(graph_us(torch, lambda: [W.sparse_matvec(layers[l].wt_down, *sel_d[l], ws=mws,
+                                                                    status=status, y=ydn[l]) for l in range(L)],
+                                    nsteps)) / L
+    matvec_bs1 = {
+        "gate_4096x11008_k%d" % kg: dict(_frac(kg * FFN * 2 + kg * 8 + FFN * 4, us_mg, peak), us_per_call=us_mg),
+        "down_11008x4096_k%d" % kd: dict(_frac(kd * D * 2 + kd * 8 + D * 4, us_md, peak), us_per_call=us_md),
+        "kernel": "k_sparse_matvec (split-K over all SMs, fixed-order partial sums)"}
+    del sel_g, sel_d, yg, ydn, mws
 
     # several tokens (the batched path): 16 tokens per call on the same layers; effective
     # bytes count the union of each projection's kept rows over the tokens
@@ -459,32 +601,18 @@ def main():
         for l in range(L):
             W.sparse_ffn_swiglu(layers[l], xbs[l], W.GATE_TOPK, kg, kg, kd, ws=wsb, status=status, y=yb)
 
-    for _ in range(3):
-        batched_step()
     union_bytes = 0
     for l in range(L):  # the kept sets of every layer (read back from the call's own views)
         W.sparse_ffn_swiglu(layers[l], xbs[l], W.GATE_TOPK, kg, kg, kd, ws=wsb, status=status, y=yb)
         v = W.ffn_ws_view(wsb, D, FFN, BT)
         ug, uu, ud = (int(v[k].bool().any(0).sum().item()) for k in ("keep_gate", "keep_up", "keep_down"))
         union_bytes += (ug + uu) * FFN * 2 + ud * D * 2 + BT * (D * 2 + D * 4) + (2 * D + FFN) * 4
-    nb_steps = max(3, args.steps // 2)
-    barrier()
-    torch.cuda.synchronize()
-    t_b0 = torch.cuda.Event(enable_timing=True)
-    t_b1 = torch.cuda.Event(enable_timing=True)
-    t_b0.record(stream)
-    for _ in range(nb_steps):
-        batched_step()
-    t_b1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    batched_ms = max_over_ranks(t_b0.elapsed_time(t_b1))
+    us_b = max_over_ranks(graph_us(torch, batched_step, nsteps)) / L
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the batched run")
-    batched = {"batch": BT, "us_per_layer": batched_ms / nb_steps * 1e3 / L,
-               "effective_gbs": world * union_bytes * nb_steps / (batched_ms * 1e-3) / 1e9,
-               "union_bytes_per_layer": union_bytes // L,
-               "path": "batched calls: select, union-row tcgen05 product, silu*mul (per projection), eager"}
+    batched = dict(_frac(union_bytes / L, us_b, peak), batch=BT, us_per_layer=us_b,
+                   union_bytes_per_layer=union_bytes // L,
+                   path="batched calls: select, union-row tcgen05 product, silu*mul (per projection)")
     del xbs, yb, wsb
 
     # end to end through the C ABI: host x in pinned memory -> device, the call, y -> host
@@ -517,16 +645,15 @@ def main():
     # the other configurations of the scope table, measured on the same GPU (each guarded:
     # a failure is reported in its entry and never affects the headline line)
     extra = {}
-    try:
-        extra["spark_ffn_gemma2_2b_bs1"] = measure_spark_ffn(W, torch, stream, max(3, args.steps // 2))
-    except Exception as e:  # pragma: no cover - reported, not raised
-        extra["spark_ffn_gemma2_2b_bs1"] = {"error": f"{type(e).__name__}: {e}"}
-    try:
-        extra["ultrasparse_down_b256"] = measure_ultrasparse(W, torch, stream, max(3, args.steps // 2))
-    except Exception as e:  # pragma: no cover
-        extra["ultrasparse_down_b256"] = {"error": f"{type(e).__name__}: {e}"}
+    for name, fn in (("spark_ffn_gemma2_2b", lambda: measure_spark(W, torch, nsteps, peak)),
+                     ("ultrasparse_down_b256", lambda: measure_ultrasparse(W, torch, nsteps, peak)),
+                     ("llama3_8b_layer", lambda: measure_llama3_layer(W, torch, nsteps, peak))):
+        try:
+            extra[name] = fn()
+        except Exception as e:  # pragma: no cover - reported, not raised
+            extra[name] = {"error": f"{type(e).__name__}: {e}"}
+        torch.cuda.empty_cache()
 
-    peak, peak_kind = _peaks()
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
     traffic = None  # ncu dram bytes of one launch, valid only for the kernel it was taken on
     tf = os.path.join(ROOT, "profiles", "ffn_fused_llama7b_traffic.txt")
@@ -547,7 +674,11 @@ def main():
                      "kernel_us": kern_ms * 1e3, "timing": "CUDA graph of the L-layer step, events around K replays"},
         "eager": {"us_per_layer": eager_ms / max(3, args.steps // 2) * 1e3 / L,
                   "kernel_us_events": eager_kern_ms * 1e3},
-        "dense": {"us_per_layer": us_layer_dense, "speedup": us_layer_dense / us_layer},
+        "dense": dict(_frac(dense_bytes, us_layer_dense, peak), us_per_layer=us_layer_dense,
+                      speedup=us_layer_dense / us_layer, kernel="wina_dense_ffn_swiglu (output-major weights)",
+                      decode_kernel_dense_mode_us=us_layer_dense_mode),
+        "p065": p065,
+        "sparse_matvec_bs1": matvec_bs1,
         "batched": batched,
         "other_configs": extra,
         "e2e": {"value": e2e_gbs, "unit": "GB/s", "us_per_layer": e2e_ms / args.steps * 1e3 / L,
@@ -572,7 +703,7 @@ def main():
 def _kernel_sha() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("common.cuh", "ffn_decode.cu"):
+    for f in ("common.cuh", "regsel.cuh", "ffn_decode.cu"):
         with open(os.path.join(ROOT, "free_activation_sparse_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
