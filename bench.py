@@ -542,15 +542,19 @@ def main():
     peak, peak_kind = _peaks()
     nsteps = max(3, args.steps // 2)
 
-    # dense comparator: the unsparsified FFN on the output-major weights (dedicated dense
-    # GEMV kernels: one warp per output row, no selection, no cross-CTA sums)
-    dbuf = torch.empty(D + FFN, dtype=torch.float32, device="cuda")
+    # dense comparator: the unsparsified FFN on the output-major weights (one cooperative
+    # launch streaming the weights as flat slab ranges, no selection)
+    dws = W.Workspace(W.OP_DENSE_FFN, D, FFN, 0, 1)
+    dst = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def dense_step():
         for l in range(L):
-            W.dense_ffn_swiglu(outmajor[l][0], outmajor[l][1], outmajor[l][2], xs[l][0], y=ys[l][0], buf=dbuf)
+            W.dense_ffn_swiglu(outmajor[l][0], outmajor[l][1], outmajor[l][2], xs[l][0], y=ys[l][0], ws=dws,
+                               status=dst)
 
     us_layer_dense = max_over_ranks(graph_us(torch, dense_step, nsteps)) / L
+    if int(dst.item()) != 0:
+        raise RuntimeError(f"dense comparator: device status {int(dst.item())}")
     dense_bytes = 3 * D * FFN * 2 + D * 2 + D * 4
     # the decode kernel itself with every channel kept (its own dense mode)
     us_layer_dense_mode = max_over_ranks(graph_us(torch, lambda: step(W.GATE_DENSE), nsteps)) / L

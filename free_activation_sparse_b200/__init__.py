@@ -30,7 +30,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_DTYPE, ERR_WORKSPACE, ERR_CAPACITY, ERR_CUD
 F32, BF16 = 0, 1
 LAYOUT_OUT_IN, LAYOUT_IN_MAJOR = 0, 1
 GATE_TOPK, GATE_STAT, GATE_DENSE = 0, 1, 2
-OP_SELECT_TOPK, OP_STAT_THRESHOLD, OP_SPARSE_MATVEC, OP_FFN_SWIGLU, OP_SPARK_FFN = 0, 1, 2, 3, 4
+OP_SELECT_TOPK, OP_STAT_THRESHOLD, OP_SPARSE_MATVEC, OP_FFN_SWIGLU, OP_SPARK_FFN, OP_DENSE_FFN = 0, 1, 2, 3, 4, 5
 
 
 class WinaError(RuntimeError):
@@ -74,7 +74,7 @@ def _load() -> ctypes.CDLL:
         "sparse_ffn_swiglu": (E, [ctypes.POINTER(_FfnT), P, E, I64, E, I64, I64, I64, D, P, P, SZ, P, P]),
         "wina_dense_matvec": (E, [P, E, I64, I64, P, E, P, P, P]),
         "spark_ffn_swiglu": (E, [P, P, P, E, I64, I64, P, E, D, P, P, P, P, P, SZ, P, P]),
-        "wina_dense_ffn_swiglu": (E, [P, P, P, E, I64, I64, P, E, P, P, P]),
+        "wina_dense_ffn_swiglu": (E, [P, P, P, E, I64, I64, P, E, P, P, SZ, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -343,7 +343,7 @@ def dense_matvec(W, x, y=None, xbuf=None):
     return y
 
 
-def dense_ffn_swiglu(W_gate, W_up, W_down, x, y=None, buf=None):
+def dense_ffn_swiglu(W_gate, W_up, W_down, x, y=None, ws: Workspace | None = None, status=None):
     """The dense comparator of the FFN on the output-major weights (one token): returns y [d]."""
     torch = _torch()
     for t_, nm in ((W_gate, "W_gate"), (W_up, "W_up"), (W_down, "W_down"), (x, "x")):
@@ -351,10 +351,11 @@ def dense_ffn_swiglu(W_gate, W_up, W_down, x, y=None, buf=None):
     ffn, d = W_gate.shape
     if y is None:
         y = torch.empty(d, dtype=torch.float32, device=x.device)
-    if buf is None:
-        buf = torch.empty((d + 3) // 4 * 4 + ffn, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = Workspace(OP_DENSE_FFN, d, ffn, 0, 1, device=x.device)
     _check(lib.wina_dense_ffn_swiglu(_ptr(W_gate), _ptr(W_up), _ptr(W_down), _dt(W_gate), d, ffn, _ptr(x), _dt(x),
-                                     _ptr(y), _ptr(buf), _stream()), "wina_dense_ffn_swiglu")
+                                     _ptr(y), ws.ptr, ws.nbytes, _ptr(status) if status is not None else None,
+                                     _stream()), "wina_dense_ffn_swiglu")
     return y
 
 

@@ -73,21 +73,28 @@ cudaError_t ensure_smem_limit(const void* kern, size_t smem) {
   return cudaSuccess;
 }
 
-cudaError_t ensure_prefer_l1(const void* kern) {
+cudaError_t ensure_carveout(const void* kern, int pct) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     for (int i = 0; i < g_nl1; ++i)
-      if (g_l1[i].dev == dev && g_l1[i].kern == kern) return cudaSuccess;
+      if (g_l1[i].dev == dev && g_l1[i].kern == kern && g_l1[i].smem == (size_t)pct) return cudaSuccess;
   }
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxL1);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (g_nl1 < kCacheSlots) g_l1[g_nl1++] = SmemEntry{dev, kern, 0};
+  for (int i = 0; i < g_nl1; ++i)
+    if (g_l1[i].dev == dev && g_l1[i].kern == kern) {
+      g_l1[i].smem = (size_t)pct;
+      return cudaSuccess;
+    }
+  if (g_nl1 < kCacheSlots) g_l1[g_nl1++] = SmemEntry{dev, kern, (size_t)pct};
   return cudaSuccess;
 }
+
+cudaError_t ensure_prefer_l1(const void* kern) { return ensure_carveout(kern, (int)cudaSharedmemCarveoutMaxL1); }
 
 int blocks_per_sm(const void* kern, int threads, size_t smem) {
   int dev = 0;
@@ -171,6 +178,7 @@ extern "C" size_t wina_workspace_size(wina_op_t op, int64_t n, int64_t m, int64_
     case WINA_OP_SPARSE_MATVEC: return spmv_total_ws(n, m, batch);
     case WINA_OP_FFN_SWIGLU: return ffn_ws_layout(n, m, batch).total;
     case WINA_OP_SPARK_FFN: return batch == 1 ? spark_ws_size(n, m) : 0;
+    case WINA_OP_DENSE_FFN: return batch == 1 ? dense_ws_size(n, m) : 0;
     default: return 0;
   }
 }

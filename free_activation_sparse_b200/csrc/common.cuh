@@ -409,40 +409,22 @@ __device__ void hist_crossing(const uint32_t* __restrict__ hist, uint32_t r, uin
 // one-pass mean / variance (Welford per thread, Chan's pairwise merge across threads)
 // ------------------------------------------------------------------------------------
 
-struct Moments {
-  double n, mean, m2;
-};
-
-__device__ __forceinline__ Moments merge_moments(Moments a, Moments b) {
-  if (b.n == 0.0) return a;
-  if (a.n == 0.0) return b;
-  const double n = a.n + b.n;
-  const double d = b.mean - a.mean;
-  return Moments{n, a.mean + d * (b.n / n), a.m2 + b.m2 + d * d * (a.n * b.n / n)};
-}
-
-// Block-wide merge in a fixed tree order (deterministic). `red` SMEM of >= 3*NT/32
-// doubles. All threads receive the result.
+// Block-wide sum of one double per thread in a fixed order: a shuffle tree inside each
+// warp, then the warps' sums by a butterfly in which every pairwise add is commutative, so
+// that all threads receive the same bits. `red` SMEM of >= NT/32 doubles. Contains two
+// __syncthreads.
 template <int NT>
-__device__ Moments block_moments(Moments m, double* red) {
+__device__ __forceinline__ double block_sum_f64(double v, double* red) {
   constexpr int NW = NT / 32;
+  static_assert(NW <= 32, "one warp combines the warps' sums");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    Moments o_;
-    o_.n = __shfl_down_sync(0xffffffffu, m.n, o);
-    o_.mean = __shfl_down_sync(0xffffffffu, m.mean, o);
-    o_.m2 = __shfl_down_sync(0xffffffffu, m.m2, o);
-    m = merge_moments(m, o_);
-  }
-  if (lane == 0) {
-    red[warp] = m.n;
-    red[NW + warp] = m.mean;
-    red[2 * NW + warp] = m.m2;
-  }
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+  if (lane == 0) red[warp] = v;
   __syncthreads();
-  Moments t{0.0, 0.0, 0.0};
-  for (int w = 0; w < NW; ++w) t = merge_moments(t, Moments{red[w], red[NW + w], red[2 * NW + w]});
+  double t = lane < NW ? red[lane] : 0.0;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
   __syncthreads();
   return t;
 }

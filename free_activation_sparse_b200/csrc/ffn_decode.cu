@@ -120,24 +120,28 @@ __device__ __forceinline__ void dcta_time(unsigned long long* t, int i) {
   if (threadIdx.x == 0) t[blockIdx.x * 4 + i] = globaltimer_ns();
 }
 
+// Spark's statistical threshold on the CTA's n values (thread t holds v[i] = element
+// t + i * kDT): mu = mean, sigma^2 = mean of (v - mu)^2 (two passes over the registers,
+// float64 sums), kept = v > mu + sigma z, as flag words.
 template <int KMAX>
 __device__ __forceinline__ void flags_from_stat(const float (&v)[KMAX], int kpt, int n, double z,
                                                 uint32_t* flags) {
-  __shared__ double dred[3 * kDW];
+  __shared__ double dred[kDW];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  Moments mo{0.0, 0.0, 0.0};
+  double s = 0.0;
 #pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
+  for (int i = 0; i < KMAX; ++i)
+    if (i < kpt && t + i * kDT < n) s += (double)v[i];
+  const double mu = block_sum_f64<kDT>(s, dred) / (double)n;
+  double q = 0.0;
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i)
     if (i < kpt && t + i * kDT < n) {
-      const double f = (double)v[i];
-      mo.n += 1.0;
-      const double dl = f - mo.mean;
-      mo.mean += dl / mo.n;
-      mo.m2 += dl * (f - mo.mean);
+      const double dl = (double)v[i] - mu;
+      q += dl * dl;
     }
-  }
-  const Moments tot = block_moments<kDT>(mo, dred);
-  const double th = tot.mean + sqrt(tot.m2 / (double)n) * z;
+  const double var = block_sum_f64<kDT>(q, dred) / (double)n;
+  const double th = mu + sqrt(var) * z;
 #pragma unroll
   for (int i = 0; i < KMAX; ++i) {
     if (i < kpt) {

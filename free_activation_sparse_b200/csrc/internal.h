@@ -41,6 +41,8 @@ cudaError_t ensure_smem_limit(const void* kern, size_t smem);
 // Ask for the smallest shared-memory carveout (the rest of the SM's unified L1/SMEM stays
 // L1) for `kern` on the current device (remembered per device and kernel).
 cudaError_t ensure_prefer_l1(const void* kern);
+// Shared-memory carveout preference of a kernel, in percent of the maximum (cached).
+cudaError_t ensure_carveout(const void* kern, int pct);
 
 // Co-resident CTAs per SM of `kern` at this block size and SMEM on the current device
 // (cached per device, kernel, block size and SMEM). 0 on error.
@@ -178,6 +180,7 @@ wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m
 wina_status_t launch_silu_mul(const float* g, const float* u, float* h, int64_t count, cudaStream_t s);
 // Workspace bytes of spark_ffn_swiglu (spark.cu).
 size_t spark_ws_size(int64_t d, int64_t ffn);
+size_t dense_ws_size(int64_t d, int64_t ffn);
 // The union path (union_gemm.cu); ws is the union region of the workspace.
 wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const int32_t* idx, const float* xs, int k,
                                   const int32_t* count, int ld, int batch, float* y, void* ws, int32_t* status,

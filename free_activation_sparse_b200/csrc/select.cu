@@ -99,22 +99,24 @@ __global__ void __launch_bounds__(NT) k_stat_threshold(const void* __restrict__ 
                                                        int32_t* __restrict__ count, float* __restrict__ tout, int cap,
                                                        int32_t* status) {
   extern __shared__ __align__(16) float vals[];  // [n]
-  __shared__ double dred[3 * NT / 32];
+  __shared__ double dred[NT / 32];
   __shared__ uint32_t wsm[2 * NT / 32 + 1];
   const int64_t b = blockIdx.x;
   const int64_t off = b * (int64_t)n;
-  Moments mo{0.0, 0.0, 0.0};
+  // mu = mean, sigma^2 = mean of (v - mu)^2: two passes, float64 sums in a fixed order
+  double s = 0.0;
   for (int i = threadIdx.x; i < n; i += NT) {
     const float f = load_elem(v, vdt, off + i);
     vals[i] = f;
-    mo.n += 1.0;
-    const double dl = (double)f - mo.mean;
-    mo.mean += dl / mo.n;
-    mo.m2 += dl * ((double)f - mo.mean);
+    s += (double)f;
   }
-  const Moments tot = block_moments<NT>(mo, dred);  // contains __syncthreads
-  const double mu = tot.mean;
-  const double var = tot.m2 / (double)n;
+  const double mu = block_sum_f64<NT>(s, dred) / (double)n;  // contains __syncthreads
+  double q = 0.0;
+  for (int i = threadIdx.x; i < n; i += NT) {
+    const double dl = (double)vals[i] - mu;
+    q += dl * dl;
+  }
+  const double var = block_sum_f64<NT>(q, dred) / (double)n;
   const double t = mu + sqrt(var) * z;
   const int64_t ob = b * (int64_t)cap;
   const uint32_t total = compact_pred<NT>(

@@ -69,7 +69,8 @@ static SparkWs spark_ws_layout(int64_t d, int64_t ffn) {
 
 size_t spark_ws_size(int64_t d, int64_t ffn) { return spark_ws_layout(d, ffn).total; }
 
-wina_status_t launch_dense_gemv(const void* W, int wdt, int m, int n, const float* xf, float* y, cudaStream_t s);
+wina_status_t launch_dense_gemv(const void* W, int wdt, int m, int n, const void* x, int xdt, float* y, float* xbuf,
+                                cudaStream_t s);
 wina_status_t launch_widen(const void* x, int xdt, int n, float* xf, cudaStream_t s);
 
 }  // namespace wina
@@ -98,8 +99,8 @@ extern "C" wina_status_t spark_ffn_swiglu(const void* W_gate, const void* W_up, 
   float* h = reinterpret_cast<float*>(w + L.h);
   cudaStream_t st = (cudaStream_t)stream;
   wina_status_t r;
-  if ((r = launch_widen(x, xdt, (int)d, xf, st))) return r;
-  if ((r = launch_dense_gemv(W_gate, wdt, (int)ffn, (int)d, xf, g, st))) return r;
+  if ((r = launch_widen(x, xdt, (int)d, xf, st))) return r;  // for the up rows
+  if ((r = launch_dense_gemv(W_gate, wdt, (int)ffn, (int)d, x, xdt, g, xf, st))) return r;
   const double z = wina_normal_quantile(1.0 - s);
   if ((r = launch_stat_threshold(g, WINA_F32, (int)ffn, z, 1, idx, nullptr, count, nullptr, (int)ffn, status_dev, st)))
     return r;

@@ -81,7 +81,8 @@ typedef enum {
   WINA_OP_STAT_THRESHOLD = 1,
   WINA_OP_SPARSE_MATVEC = 2,
   WINA_OP_FFN_SWIGLU = 3,
-  WINA_OP_SPARK_FFN = 4
+  WINA_OP_SPARK_FFN = 4,
+  WINA_OP_DENSE_FFN = 5
 } wina_op_t;
 
 /* The three projections of a SwiGLU FFN, already packed input-major:
@@ -157,6 +158,7 @@ double wina_normal_quantile(double p);
  *                          batch = tokens.
  *   WINA_OP_FFN_SWIGLU:    n = d, m = ffn, k ignored, batch = tokens.
  *   WINA_OP_SPARK_FFN:     n = d, m = ffn, k ignored, batch = 1.
+ *   WINA_OP_DENSE_FFN:     n = d, m = ffn, k ignored, batch = 1.
  *   WINA_OP_SELECT_TOPK, WINA_OP_STAT_THRESHOLD: 0.                                  */
 size_t wina_workspace_size(wina_op_t op, int64_t n, int64_t m, int64_t k, int64_t batch);
 
@@ -311,22 +313,39 @@ wina_status_t spark_ffn_swiglu(const void* W_gate, const void* W_up, const void*
                                int32_t* status_dev, wina_stream_t stream);
 
 /* The dense comparator: the unsparsified layer y = W x (every channel kept), on the
- * OUTPUT-major weight W[m][n] (the matrix that multiplies x, unpacked), one warp per output
- * row with 16-byte streaming loads; no workspace beyond xbuf. Batch 1.
- *   W:    device [m][n] of wdt (n % 8 == 0 for bf16, % 4 for f32).
+ * OUTPUT-major weight W[m][n] (the matrix that multiplies x, unpacked). The weights are
+ * streamed as one flat sequence of 512-byte slabs split evenly over all warps, x staged in
+ * shared memory; a row split between two warps is completed by two atomic adds onto a
+ * zeroed y, which gives the same bits in either order. Batch 1. Rows that are not a whole
+ * number of slabs (n not a multiple of 256 for bf16, 128 for f32), or whose x does not fit
+ * in 96 KB of shared memory, take a warp-per-row kernel that reads x through L1.
+ *   W:    device [m][n] of wdt (n % 8 == 0 for bf16, % 4 for f32), 16-byte aligned.
  *   x:    device [n] of xdt.   y: device float32 [m] (written).
- *   xbuf: device float32 [n] scratch (x widened), 16-byte aligned. */
+ *   xbuf: device float32 [n] scratch (x widened; used by the long-row kernel only),
+ *         16-byte aligned. */
 wina_status_t wina_dense_matvec(const void* W, wina_dtype_t wdt, int64_t m, int64_t n, const void* x,
                                 wina_dtype_t xdt, float* y, float* xbuf, wina_stream_t stream);
 
 /* The dense comparator of sparse_ffn_swiglu: y = W_down (silu(W_gate x) * (W_up x)) with
  * every channel kept, on the output-major weights W_gate, W_up [ffn][d] and W_down
- * [d][ffn]. Two launches: gate and up rows together (h), then down. Batch 1.
+ * [d][ffn]. One cooperative launch of two 512-thread CTAs per SM: W_gate streamed into g
+ * by half of the warps and W_up into u by the other half, each as equal flat ranges of
+ * 512-byte slabs (by atomic adds, at most two per element, so the bits do not depend on
+ * timing), y zeroed on the way; a grid barrier, with the first down loads already in
+ * flight; h = silu(g) * u staged by every CTA in shared memory; W_down streamed into y.
+ * g and u live in one of two workspace copies used by alternate calls: each call zeroes
+ * the copy the next call adds into.
+ * Rows that are not a whole number of slabs (d or ffn not a multiple of 256 for bf16, 128
+ * for f32), or whose x or h does not fit in 96 KB of shared memory, take three
+ * warp-per-row launches instead. Batch 1.
  *   x: device [d] of xdt;  y: device float32 [d] (written);
- *   buf: device float32 scratch of round_up(d, 4) + ffn floats, 16-byte aligned. */
+ *   ws: device scratch of at least wina_workspace_size(WINA_OP_DENSE_FFN, d, ffn, 0, 1)
+ *       bytes, zero-filled before first use (it holds the grid barrier), 16-byte aligned;
+ *   status_dev: optional device int32; WINA_ERR_TIMEOUT is recorded there if a grid
+ *       barrier wait runs out (y is then incomplete and ws must be zero-filled again). */
 wina_status_t wina_dense_ffn_swiglu(const void* W_gate, const void* W_up, const void* W_down, wina_dtype_t wdt,
-                                    int64_t d, int64_t ffn, const void* x, wina_dtype_t xdt, float* y, float* buf,
-                                    wina_stream_t stream);
+                                    int64_t d, int64_t ffn, const void* x, wina_dtype_t xdt, float* y, void* ws,
+                                    size_t ws_bytes, int32_t* status_dev, wina_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -58,6 +58,9 @@ def test_workspace_sizes():
     f8 = W.workspace_size(W.OP_FFN_SWIGLU, 4096, 11008, 0, 8)
     assert f8 > f4 >= 4 * (2 * 4096 + 11008) * 8  # several tokens: per-token index and value lists
     assert W.workspace_size(W.OP_SELECT_TOPK, 10, 10, 1, 1) == 0
+    dn = W.workspace_size(W.OP_DENSE_FFN, 4096, 11008, 0, 1)
+    assert dn >= 128 + 2 * 11008 * 4  # barrier, g, u
+    assert W.workspace_size(W.OP_DENSE_FFN, 4096, 11008, 0, 2) == 0  # one token
     assert W.workspace_size(W.OP_FFN_SWIGLU, 0, 10, 0, 1) == 0
 
 
