@@ -7,3 +7,4 @@ library and does not import it.
 """
 
 from .wina_oracle import *  # noqa: F401,F403
+from .ds_oracle import *  # noqa: F401,F403
