@@ -19,7 +19,8 @@ __all__ = [
     "abi_version", "normal_quantile", "workspace_size", "Workspace", "FfnWeights",
     "pack_in_major", "col_norms", "select_topk", "stat_topk_threshold", "sparse_matvec",
     "sparse_ffn_swiglu", "ffn_ws_view", "ffn_prepare", "declared_symbols", "sparse_matvec_noalloc",
-    "dense_matvec", "dense_ffn_swiglu", "spark_ffn",
+    "dense_matvec", "dense_ffn_swiglu", "spark_ffn", "ds_channel_absmean", "ds_calibrate_channels",
+    "ds_label_build", "ds_decode_attention",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwina.so")
@@ -75,6 +76,11 @@ def _load() -> ctypes.CDLL:
         "wina_dense_matvec": (E, [P, E, I64, I64, P, E, P, P, P]),
         "spark_ffn_swiglu": (E, [P, P, P, E, I64, I64, P, E, D, P, P, P, P, P, SZ, P, P]),
         "wina_dense_ffn_swiglu": (E, [P, P, P, E, I64, I64, P, E, P, P, SZ, P, P]),
+        "ds_channel_absmean": (E, [P, E, I64, I64, I64, I64, P, P, P]),
+        "ds_label_build": (E, [P, E, I64, I64, I64, I64, P, P, I64, I64, I64, P, P]),
+        "ds_decode_smem_bytes": (SZ, [I64, I64, I64]),
+        "ds_decode_attention": (E, [P, E, P, P, P, E, P, I64, I64, I64, I64, I64, I64, P, I64, ctypes.c_float, P, P, P,
+                                    P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -402,3 +408,67 @@ def ffn_ws_view(ws: Workspace, d: int, ffn: int, batch: int) -> dict:
         stamps=take(v.stamps, 16, torch.int64, (16,)),
         cta_t=take(v.cta_t, 296 * 4, torch.int64, (296, 4)),
     )
+
+
+# ------------------------------------------------------------------------------------
+# Double Sparsity decode attention
+# ------------------------------------------------------------------------------------
+
+
+def ds_channel_absmean(K, seq_len):
+    """Mean |K| per (key/value head, channel) over the valid tokens: K [B][Hkv][Tmax][dh],
+    seq_len int32 [B] -> float32 [Hkv][dh]."""
+    torch = _torch()
+    _cuda(K, "K")
+    _cuda(seq_len, "seq_len")
+    B, Hkv, Tmax, dh = K.shape
+    out = torch.empty((Hkv, dh), dtype=torch.float32, device=K.device)
+    _check(lib.ds_channel_absmean(_ptr(K), _dt(K), B, Hkv, Tmax, dh, _ptr(seq_len), _ptr(out), _stream()),
+           "ds_channel_absmean")
+    return out
+
+
+def ds_calibrate_channels(K, seq_len, r: int):
+    """The K-outlier channels: the r channels of largest mean |K| per key/value head,
+    ascending (int32 [Hkv][r]); the means go through the top-K gate kernel."""
+    a = ds_channel_absmean(K, seq_len)
+    idx, _ = select_topk(a, None, r)
+    return idx
+
+
+def ds_label_build(K, seq_len, channels, t0: int = 0, t1: int | None = None, label=None):
+    """The label cache [B][Hkv][Tmax][r] (K's dtype) for tokens [t0, t1)."""
+    torch = _torch()
+    for t_, nm in ((K, "K"), (seq_len, "seq_len"), (channels, "channels")):
+        _cuda(t_, nm)
+    B, Hkv, Tmax, dh = K.shape
+    r = channels.shape[1]
+    if t1 is None:
+        t1 = Tmax
+    if label is None:
+        label = torch.zeros((B, Hkv, Tmax, r), dtype=K.dtype, device=K.device)
+    _check(lib.ds_label_build(_ptr(K), _dt(K), B, Hkv, Tmax, dh, _ptr(seq_len), _ptr(channels), r, t0, t1,
+                              _ptr(label), _stream()), "ds_label_build")
+    return label
+
+
+def ds_decode_attention(q, K, V, label, channels, seq_len, k: int, scale: float = 0.0, out=None,
+                        want_idx: bool = False, want_scores: bool = False, status=None):
+    """One Double Sparsity decode step: q [B][Hq][dh] -> out float32 [B][Hq][dh]; with
+    want_idx / want_scores also the kept tokens [B][Hq][k] and the approximate scores
+    [B][Hq][Tmax]. Returns (out, idx or None, scores or None)."""
+    torch = _torch()
+    for t_, nm in ((q, "q"), (K, "K"), (V, "V"), (label, "label"), (channels, "channels"), (seq_len, "seq_len")):
+        _cuda(t_, nm)
+    B, Hq, dh = q.shape
+    _, Hkv, Tmax, _ = K.shape
+    r = channels.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, dh), dtype=torch.float32, device=q.device)
+    idx = torch.full((B, Hq, k), -1, dtype=torch.int32, device=q.device) if want_idx else None
+    sc = torch.zeros((B, Hq, Tmax), dtype=torch.float32, device=q.device) if want_scores else None
+    _check(lib.ds_decode_attention(_ptr(q), _dt(q), _ptr(K), _ptr(V), _ptr(label), _dt(K), _ptr(channels), B, Hq,
+                                   Hkv, Tmax, dh, r, _ptr(seq_len), k, float(scale), _ptr(out),
+                                   _ptr(idx) if idx is not None else None, _ptr(sc) if sc is not None else None,
+                                   _ptr(status) if status is not None else None, _stream()), "ds_decode_attention")
+    return out, idx, sc

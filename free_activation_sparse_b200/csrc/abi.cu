@@ -105,7 +105,7 @@ int blocks_per_sm(const void* kern, int threads, size_t smem) {
       if (g_occ[i].dev == dev && g_occ[i].kern == kern && g_occ[i].threads == threads && g_occ[i].smem == smem)
         return g_occ[i].per_sm;
   }
-  if (smem > 48 * 1024 && ensure_smem_limit(kern, smem) != cudaSuccess) return 0;
+  if (ensure_smem_limit(kern, smem) != cudaSuccess) return 0;  // static shared memory comes on top
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lk(g_mu);

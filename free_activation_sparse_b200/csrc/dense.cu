@@ -377,7 +377,7 @@ template <bool BF16, int U>
 static wina_status_t launch_slabs(const void* W, int m, int n, const void* x, int xdt, float* y, cudaStream_t s) {
   const void* kern = (const void*)k_dense_slabs<BF16, U>;
   const size_t smem = slab_smem(n, VecOps<BF16>::EPV);
-  if (smem > 48 * 1024) {
+  {  // always: static shared memory comes on top of the dynamic part
     const cudaError_t e = ensure_smem_limit(kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
   }
@@ -447,7 +447,7 @@ static wina_status_t launch_dense_ffn_fused(const DenseFfnParams& p0, bool bf16,
     return WINA_ERR_UNSUPPORTED_DTYPE;
   void* kern = bf16 ? (void*)k_dense_ffn<true> : (void*)k_dense_ffn<false>;
   const size_t smem = std::max(slab_smem(p0.d, epv), slab_smem(p0.ffn, epv));
-  if (smem > 48 * 1024) {
+  {  // always: static shared memory comes on top of the dynamic part
     const cudaError_t e = ensure_smem_limit(kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
   }

@@ -612,7 +612,7 @@ wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (smem > 48 * 1024) {
+  {  // always: static shared memory comes on top of the dynamic part
     cudaError_t e = ensure_smem_limit(kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
   }

@@ -53,7 +53,7 @@ int blocks_per_sm(const void* kern, int threads, size_t smem);
 template <typename... Exp, typename... Act>
 cudaError_t launch_kernel(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool coop,
                           Act&&... args) {
-  if (smem > 48 * 1024) {
+  if (smem > 0) {  // any dynamic part: static shared memory comes on top of it
     cudaError_t e = ensure_smem_limit((const void*)kern, smem);
     if (e != cudaSuccess) return e;
   }

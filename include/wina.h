@@ -347,6 +347,55 @@ wina_status_t wina_dense_ffn_swiglu(const void* W_gate, const void* W_up, const 
                                     int64_t d, int64_t ffn, const void* x, wina_dtype_t xdt, float* y, void* ws,
                                     size_t ws_bytes, int32_t* status_dev, wina_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * Double Sparsity decode attention ("大模型DoubleSparse稀疏化技术原理", section 技术原理:
+ * 离线校准 and 在线前向计算). Caches are [B][Hkv][Tmax][dh] (keys, values) and
+ * [B][Hkv][Tmax][r] (labels), in the key cache's dtype (bf16 or f32), token t of sequence
+ * b valid for t < seq_len[b]; channels is [Hkv][r] int32 (the important channels of each
+ * key/value head, ascending). All pointers are device pointers owned by the caller.
+ * --------------------------------------------------------------------------------- */
+
+/* Offline calibration, K-outlier strategy: absmean[g][c] = mean over every sequence's
+ * valid tokens of |K[b][g][t][c]| (float64 sums, rounded once to float32). The r
+ * channels of largest mean are then picked per head with wina_select_topk(absmean, NULL
+ * c, n = dh, k = r, batch = Hkv), which lists them ascending, ties to the lower channel.
+ *   seq_len: device int32 [B];  absmean: device float32 [Hkv][dh] (written). */
+wina_status_t ds_channel_absmean(const void* K, wina_dtype_t kdt, int64_t B, int64_t Hkv, int64_t Tmax, int64_t dh,
+                                 const int32_t* seq_len, float* absmean, wina_stream_t stream);
+
+/* The label cache: label[b][g][t][j] = K[b][g][t][channels[g][j]] for t0 <= t < t1 and
+ * t < seq_len[b] (a prefill passes [0, T), a decode step the new token [T-1, T)); other
+ * entries are left as they are. 0 <= t0 <= t1 <= Tmax, 1 <= r <= dh. */
+wina_status_t ds_label_build(const void* K, wina_dtype_t kdt, int64_t B, int64_t Hkv, int64_t Tmax, int64_t dh,
+                             const int32_t* seq_len, const int32_t* channels, int64_t r, int64_t t0, int64_t t1,
+                             void* label, wina_stream_t stream);
+
+/* Bytes of dynamic shared memory ds_decode_attention needs per CTA (host function): the
+ * call is refused (WINA_ERR_INVALID_ARG) above 225 KB, i.e. for Tmax + 2 min(k, Tmax)
+ * beyond about 51 K entries. */
+size_t ds_decode_smem_bytes(int64_t Tmax, int64_t dh, int64_t k);
+
+/* One decode step of Double Sparsity attention for B sequences and Hq query heads (query
+ * head h reads key/value head h / (Hq / Hkv)); one CTA per (sequence, query head):
+ *   1. q[C]: the query's important channels (C = channels[g]);
+ *   2. s_t = sum over j of q[C_j] * label[t][j] for every valid token t, in float32, each
+ *      product rounded and added in the order j = 0..r-1;
+ *   3. S = the min(k, seq_len) tokens of largest s (signed, ties to the lower token),
+ *      ascending; out = sum over t in S of p_t V[t] with p = softmax over S of
+ *      (q . K[t]) * scale (float32; scale <= 0 means 1 / sqrt(dh)).
+ *   q: device [B][Hq][dh] of qdt;  out: device float32 [B][Hq][dh] (written; zeros when
+ *   min(k, seq_len) = 0);  idx_out: optional device int32 [B][Hq][k], the first
+ *   min(k, seq_len[b]) entries written;  scores_out: optional device float32
+ *   [B][Hq][Tmax], the first seq_len[b] written.
+ *   dh in {32, 64, 128, 256}; r a multiple of 8 (bf16) or 4 (f32), r <= dh; K, V, label
+ *   16-byte aligned. A seq_len outside [0, Tmax] records WINA_ERR_INVALID_ARG in
+ *   status_dev (optional) and is clamped. Deterministic: fixed-order sums throughout. */
+wina_status_t ds_decode_attention(const void* q, wina_dtype_t qdt, const void* K, const void* V, const void* label,
+                                  wina_dtype_t kvdt, const int32_t* channels, int64_t B, int64_t Hq, int64_t Hkv,
+                                  int64_t Tmax, int64_t dh, int64_t r, const int32_t* seq_len, int64_t k,
+                                  float scale, float* out, int32_t* idx_out, float* scores_out,
+                                  int32_t* status_dev, wina_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

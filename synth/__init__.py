@@ -15,6 +15,7 @@ from .gen import (  # noqa: F401
     make_llama3_8b_layer,
     make_gemma2_2b_spark,
     make_ultrasparse_down,
+    make_ds_decode,
     make_weight,
     spark_keep_count,
 )

@@ -1,4 +1,4 @@
-"""Seeded generators for the five synthetic workloads.
+"""Seeded generators for the synthetic workloads.
 
 Every array is drawn with numpy's PCG64 (``numpy.random.default_rng``). A workload's
 draws happen in a fixed order from one generator, so a (workload, seed) pair always
@@ -195,10 +195,40 @@ def make_ultrasparse_down(seed: int = 4, batch: int = 256, nnz_frac: float = 0.0
     return dict(name="ultrasparse_down_14336x4096_b256", W=W, x=bf16_bits_from_f32(x), n=n, m=m, nnz=nnz)
 
 
+def make_ds_decode(seed: int = 5, batch: int = 1, hq: int = 32, hkv: int = 32, seq=4096, dh: int = 128,
+                   n_outlier: int = 16, outlier_scale: float = 4.0, tmax: int | None = None) -> dict:
+    """Double Sparsity decode workload (Llama-2-7B attention shapes by default: 32 query
+    and 32 key/value heads of 128 channels, 4096 cached tokens, bf16 caches).
+
+    Draw order: per key/value head g, a set O_g of ``n_outlier`` distinct channels
+    (uniform, without replacement); then K [B][Hkv][Tmax][dh] ~ N(0, 1) with the channels
+    of O_g multiplied by ``outlier_scale``; then V ~ N(0, 1); then q [B][Hq][dh] ~ N(0, 1)
+    with the channels of its key/value head's O_g multiplied by ``outlier_scale`` (so that
+    a few channels carry most of q . K, the structure the method relies on). ``seq`` is
+    one length for every sequence or a list of B lengths; cache slots past a sequence's
+    length hold draws too (they must not be read). Caches and q are bf16 bit patterns.
+    """
+    rng = np.random.default_rng(seed)
+    seq_len = np.array([seq] * batch if np.isscalar(seq) else list(seq), dtype=np.int32)
+    T = int(tmax if tmax is not None else seq_len.max())
+    outl = np.stack([np.sort(rng.choice(dh, size=n_outlier, replace=False)) for _ in range(hkv)]).astype(np.int32)
+    colscale = np.ones((hkv, dh), dtype=np.float32)
+    for g in range(hkv):
+        colscale[g, outl[g]] = outlier_scale
+    K = (rng.standard_normal((batch, hkv, T, dh), dtype=np.float32) * colscale[None, :, None, :]).astype(np.float32)
+    V = rng.standard_normal((batch, hkv, T, dh), dtype=np.float32)
+    grp = hq // hkv
+    qs = colscale[np.arange(hq) // grp]
+    q = (rng.standard_normal((batch, hq, dh), dtype=np.float32) * qs[None]).astype(np.float32)
+    return dict(name=f"ds_decode_b{batch}_h{hq}x{hkv}_t{T}_d{dh}", K=bf16_bits_from_f32(K), V=bf16_bits_from_f32(V),
+                q=bf16_bits_from_f32(q), seq_len=seq_len, outliers=outl, B=batch, Hq=hq, Hkv=hkv, Tmax=T, dh=dh)
+
+
 WORKLOADS = {
     "linear_512x256_f32": make_linear_512x256_f32,
     "llama7b_ffn_4096x11008_bf16": make_llama7b_ffn,
     "llama3_8b_layer_bf16": make_llama3_8b_layer,
     "gemma2_2b_ffn_spark_2304x9216_bf16": make_gemma2_2b_spark,
     "ultrasparse_down_14336x4096_b256": make_ultrasparse_down,
+    "ds_decode_llama2_7b_t4096": make_ds_decode,
 }
