@@ -326,6 +326,64 @@ def measure_ultrasparse(W, torch, steps: int, peak: float, copies: int = 2) -> d
                 path="wina_select_topk (nonzero set) + sparse_matvec (union of the 256 tokens' rows on tcgen05)")
 
 
+def measure_ds_decode(W, torch, steps: int, peak: float, batches=(1, 8), copies: int = 3) -> dict:
+    """Double Sparsity decode attention on Llama-2-7B attention shapes (32 query and key/
+    value heads of 128 channels, 4096 cached tokens, bf16 caches; 16 important channels
+    per head, 256 tokens kept = 1/16): per batch size, `copies` distinct caches (above L2
+    together) called in turn inside a CUDA graph. Bytes: the label rows of every token,
+    the kept tokens' key and value rows, q and the output. Also, for B = 1, the kept sets'
+    recall of the exact top-256 by the full q . K (numpy on the synthetic cache) and the
+    output's relative L2 distance from full attention over all 4096 tokens."""
+    r, k = 16, 256
+    out = {"path": "ds_label_build (prefill, untimed) + ds_decode_attention", "r": r, "k": k, "by_batch": {}}
+    for B in batches:
+        cfg = synth.make_ds_decode(batch=B)
+        Hq, Hkv, T, dh = cfg["Hq"], cfg["Hkv"], cfg["Tmax"], cfg["dh"]
+        seq = torch.from_numpy(cfg["seq_len"]).cuda()
+        C = torch.from_numpy(cfg["outliers"]).cuda()
+        sets = []
+        for c in range(copies):
+            q, K, V = (_dev_bf16(torch, cfg[n]) for n in ("q", "K", "V"))
+            if c:
+                K = K.roll(c, dims=2).contiguous()  # a distinct cache, same statistics
+                V = V.roll(c, dims=2).contiguous()
+            sets.append((q, K, V, W.ds_label_build(K, seq, C)))
+        o = torch.empty((B, Hq, dh), dtype=torch.float32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+        def step():
+            for (q, K, V, lab) in sets:
+                W.ds_decode_attention(q, K, V, lab, C, seq, k, out=o, status=st)
+
+        us = graph_us(torch, step, steps) / copies
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status {int(st.item())}")
+        nbytes = B * Hkv * T * r * 2 + B * Hq * k * dh * 2 * 2 + B * Hq * dh * (2 + 4)
+        line = dict(_frac(nbytes, us, peak), us_per_step=us, heads=Hq, tokens=T, head_dim=dh)
+        if B == 1:
+            q, K, V, lab = sets[0]
+            o1, idx, _ = W.ds_decode_attention(q, K, V, lab, C, seq, k, want_idx=True)
+            idx = idx.cpu().numpy()[0]
+            qf = synth.f32_from_bf16_bits(cfg["q"])[0].astype(np.float64)
+            Kf = synth.f32_from_bf16_bits(cfg["K"])[0].astype(np.float64)
+            Vf = synth.f32_from_bf16_bits(cfg["V"])[0].astype(np.float64)
+            rec, err = [], []
+            full_out = np.zeros((Hq, dh))
+            for h in range(Hq):
+                sc = Kf[h] @ qf[h]
+                top = np.argsort(-sc, kind="stable")[:k]
+                rec.append(len(set(top.tolist()) & set(idx[h].tolist())) / k)
+                lg = sc / np.sqrt(dh)
+                p = np.exp(lg - lg.max())
+                full_out[h] = (p / p.sum()) @ Vf[h]
+            ds_out = o1.cpu().numpy()[0].astype(np.float64)
+            line["recall_vs_exact_topk"] = float(np.mean(rec))
+            line["rel_l2_vs_full_attention"] = float(np.linalg.norm(ds_out - full_out) / np.linalg.norm(full_out))
+        out["by_batch"][str(B)] = line
+        del sets
+    return out
+
+
 def measure_llama3_layer(W, torch, steps: int, peak: float, batches=(1, 4, 16)) -> dict:
     """Llama-3-8B-shaped decoder layer (bf16): Q/K/V/O as gated sparse products (each its
     own top-K of |input * c|; Q, K, V gate the hidden state, O an independent input since
@@ -651,7 +709,8 @@ def main():
     extra = {}
     for name, fn in (("spark_ffn_gemma2_2b", lambda: measure_spark(W, torch, nsteps, peak)),
                      ("ultrasparse_down_b256", lambda: measure_ultrasparse(W, torch, nsteps, peak)),
-                     ("llama3_8b_layer", lambda: measure_llama3_layer(W, torch, nsteps, peak))):
+                     ("llama3_8b_layer", lambda: measure_llama3_layer(W, torch, nsteps, peak)),
+                     ("double_sparsity_decode_llama2_7b", lambda: measure_ds_decode(W, torch, nsteps, peak))):
         try:
             extra[name] = fn()
         except Exception as e:  # pragma: no cover - reported, not raised

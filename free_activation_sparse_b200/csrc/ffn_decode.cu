@@ -53,7 +53,7 @@ struct DecodeParams {
   float* y;
   int Gg;        // CTAs on the gate projection
   int list_cap;  // rows per CTA list
-  uint32_t sm_flags, sm_wpre, sm_lrow, sm_lval;  // SMEM offsets (the histogram is at 0)
+  uint32_t sm_flags, sm_wpre, sm_lrow;  // SMEM offsets (the histogram is at 0)
   GridBarrier* bar;
   unsigned long long wait_ns;  // time limit of each barrier wait
   float* part;      // [G][pstride] float32 partial rows (g / u in phase B, y in phase E)
@@ -68,10 +68,10 @@ struct DecodeParams {
   int32_t* status;
 };
 
-// Dynamic SMEM: hist [kSelBins + 256] | flags [nw] | word prefix [nw] | list rows [cap] |
-// list values [cap]; the group and slice reductions (red) overlay hist.
+// Dynamic SMEM: hist [kSelBins + 256] | flags [nw] | word prefix [nw] | list rows [cap];
+// the group and slice reductions (red) overlay hist.
 struct DecodeSmem {
-  uint32_t hist, flags, wpre, lrow, lval, total;
+  uint32_t hist, flags, wpre, lrow, total;
 };
 
 __host__ __device__ inline DecodeSmem decode_smem(int n_max, int cap, int red_floats) {
@@ -90,9 +90,6 @@ __host__ __device__ inline DecodeSmem decode_smem(int n_max, int cap, int red_fl
   o += nw * 4u;
   o = (o + 15u) & ~15u;
   L.lrow = o;
-  o += (uint32_t)cap * 4u;
-  o = (o + 15u) & ~15u;
-  L.lval = o;
   o += (uint32_t)cap * 4u;
   L.total = (o + 127u) & ~127u;
   return L;
@@ -203,19 +200,20 @@ __device__ int list_rows(const uint32_t* flags, int n, int parts, int part, uint
 // streaming the listed rows
 // ------------------------------------------------------------------------------------
 
-// Partial rows of one CTA's product: the two row groups of a CTA whose rows take 512
-// threads store one each; narrower rows (more groups) are summed in SMEM into one.
-__host__ __device__ inline int decode_partials(int V) { return decode_tpr(V) == kDT / 2 ? 2 : 1; }
-
-// This CTA's partial row(s) of sum over the listed rows r of lval[r] * Wt[lrow[r]][0..m),
-// read with 16-byte loads: row p = blockIdx.x * P + q (q < P = decode_partials(V)) of
-// `part` (row stride pstride floats). The CTA is split into NG = kDT / TPR groups of TPR
-// threads; group g takes list entries g, g + NG, ...; thread l of a group owns VPT vectors
-// of each row, those of index l, l + TPR, ... rotated by an offset that differs from CTA
-// to CTA, and keeps U rows in flight. With more than two groups their sums are combined in
-// SMEM (red, at least (NG - 1) * TPR * EPV floats, groups in order) before the store.
-template <bool BF16, int VPT, int U>
-__device__ void stream_rows(const void* __restrict__ Wt, int m, const int* lrow, const float* lval, int cnt,
+// This CTA's partial row(s) of sum over the listed rows r of val(lrow[r]) *
+// Wt[lrow[r]][0..m), read with 16-byte loads, stored in `part` (row stride pstride floats).
+// The CTA is split into NG = kDT / TPR groups of TPR threads; group g takes list entries
+// g, g + NG, ...; thread l of a group owns VPT vectors of each row, those of index l,
+// l + TPR, ... rotated by an offset that differs from CTA to CTA. Rows are loaded U at a
+// time, with DB into two register buffers in turn so that the next rows are in flight
+// while the current ones are multiplied; the last batch is predicated (no row-by-row
+// tail). A row's input value val(channel) is loaded with its weights. The groups' sums
+// are stored as partial rows blockIdx.x * P + g (P = decode_partials(V) = 2 when two
+// groups of 512 threads take the rows), or, with more groups, combined in SMEM in group
+// order first (red: at least (NG - 1) * TPR * EPV floats) and stored as row blockIdx.x;
+// fixed order throughout, so the result is bit-reproducible.
+template <bool BF16, int VPT, int U, bool DB, typename Val>
+__device__ void stream_rows(const void* __restrict__ Wt, int m, const int* lrow, Val val, int cnt,
                             float* __restrict__ part, int pstride, float* red, uint64_t pol, long long* stamp_loop,
                             unsigned long long* t_loop) {
   constexpr int EPV = VecOps<BF16>::EPV;
@@ -236,36 +234,53 @@ __device__ void stream_rows(const void* __restrict__ Wt, int m, const int* lrow,
   for (int j = 0; j < VPT; ++j)
 #pragma unroll
     for (int e = 0; e < EPV; ++e) acc[j][e] = 0.f;
-  int r = g;
-  for (; r + (U - 1) * NG < cnt; r += U * NG) {
-    uint4 w[U][VPT];
+  const int mine = cnt > g ? (cnt - g + NG - 1) / NG : 0;  // this group's rows
+  uint4 wa[U][VPT], wb[U][VPT];
+  float xa[U], xb[U];
+  // rows i0 .. i0 + U - 1 of this group (those below `mine`) into (w, xv)
+  auto load = [&](uint4 (&w)[U][VPT], float (&xv)[U], int i0) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const uint4* rp = base + (int64_t)lrow[r + u * NG] * V;
+      if (i0 + u < mine) {
+        const int row = lrow[g + (i0 + u) * NG];
+        xv[u] = val(row);
+        const uint4* rp = base + (int64_t)row * V;
 #pragma unroll
-      for (int j = 0; j < VPT; ++j)
-        if (vid[j] >= 0) w[u][j] = ld_stream_u4(rp + vid[j], pol);
+        for (int j = 0; j < VPT; ++j)
+          if (vid[j] >= 0) w[u][j] = ld_stream_u4(rp + vid[j], pol);
+      }
     }
+  };
+  auto consume = [&](const uint4 (&w)[U][VPT], const float (&xv)[U], int i0) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const float xv = lval[r + u * NG];
+      if (i0 + u < mine) {
 #pragma unroll
-      for (int j = 0; j < VPT; ++j)
-        if (vid[j] >= 0) VecOps<BF16>::fma(acc[j], w[u][j], xv);
+        for (int j = 0; j < VPT; ++j)
+          if (vid[j] >= 0) VecOps<BF16>::fma(acc[j], w[u][j], xv[u]);
+      }
     }
-  }
-  for (; r < cnt; r += NG) {
-    const uint4* rp = base + (int64_t)lrow[r] * V;
-    const float xv = lval[r];
-#pragma unroll
-    for (int j = 0; j < VPT; ++j)
-      if (vid[j] >= 0) VecOps<BF16>::fma(acc[j], ld_stream_u4(rp + vid[j], pol), xv);
+  };
+  if (DB) {
+    load(wa, xa, 0);
+    for (int i0 = 0; i0 < mine; i0 += 2 * U) {
+      if (i0 + U < mine) load(wb, xb, i0 + U);
+      consume(wa, xa, i0);
+      if (i0 + U >= mine) break;
+      if (i0 + 2 * U < mine) load(wa, xa, i0 + 2 * U);
+      consume(wb, xb, i0 + U);
+    }
+  } else {
+    for (int i0 = 0; i0 < mine; i0 += U) {
+      load(wa, xa, i0);
+      consume(wa, xa, i0);
+    }
   }
   if (t == 0) {
     if (blockIdx.x == 0) *stamp_loop = clock64();
     *t_loop = globaltimer_ns();
   }
-  if (NG == 2) {  // each group stores its own partial row
+  if (NG == 2) {  // each group stores its own partial row (no wait for the other group)
     float* out = part + (size_t)(blockIdx.x * 2 + g) * pstride;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
@@ -278,6 +293,7 @@ __device__ void stream_rows(const void* __restrict__ Wt, int m, const int* lrow,
     }
     return;
   }
+  // more (narrower) groups: their sums are combined in SMEM in group order first
   float* out = part + (size_t)blockIdx.x * pstride;
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
@@ -300,6 +316,10 @@ __device__ void stream_rows(const void* __restrict__ Wt, int m, const int* lrow,
   __syncthreads();  // red (which overlays the selection histogram) is free again
 }
 
+// Partial rows a CTA stores for rows of V vectors: the two row groups of a CTA whose rows
+// take 512 threads store one each; narrower rows (more groups) are summed into one.
+__host__ __device__ inline int decode_partials(int V) { return decode_tpr(V) == kDT / 2 ? 2 : 1; }
+
 // Reduce-scatter of the partial rows: for this CTA's nq (<= 32) float4 columns
 // q0 .. q0 + nq - 1, the sums over rows p in [0, split) and in [split, end) of
 // part[p][4q .. 4q + 3]. Warp w reads rows w, w + 32, ... in turn (lane i column q0 + i, so
@@ -314,7 +334,7 @@ __device__ void reduce_scatter(const float* __restrict__ part, int pstride, int 
   if (lane < nq) {
     const float4* col = reinterpret_cast<const float4*>(part) + q0 + lane;
     const int rs = pstride / 4;
-#pragma unroll 4
+#pragma unroll 8
     for (int p = warp; p < end; p += 32) {
       const float4 v = __ldcg(col + (size_t)p * rs);
       if (p < split) {  // warp-uniform
@@ -365,7 +385,6 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   uint32_t* flags = reinterpret_cast<uint32_t*>(smraw + a.sm_flags);
   uint32_t* wpre = reinterpret_cast<uint32_t*>(smraw + a.sm_wpre);
   int* lrow = reinterpret_cast<int*>(smraw + a.sm_lrow);
-  float* lval = reinterpret_cast<float*>(smraw + a.sm_lval);
   const int G = gridDim.x, b = blockIdx.x, t = threadIdx.x;
   const uint64_t pol = l2_evict_first_policy();
   const int npb = decode_partials(ffn * (int)ESZ / 16), npe = decode_partials(d * (int)ESZ / 16);
@@ -408,7 +427,6 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   }
   __syncthreads();
   int cnt = list_rows(flags, d, parts, part, wpre, lrow, a.list_cap, a.status);
-  for (int r = t; r < cnt; r += kDT) lval[r] = load_elem(a.x, a.xdt, lrow[r]);
   if (part == parts - 1) {
     uint8_t* kb = gate ? a.keep_g : a.keep_u;
     for (int j = t; j < d; j += kDT) kb[j] = (uint8_t)((flags[j >> 5] >> (j & 31)) & 1u);
@@ -418,7 +436,8 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   dcta_time(a.cta_t, 0);
 
   // ---------------- B: stream the gate / up rows into this CTA's partial row ----------------
-  stream_rows<BF16, VB, UB>(wt, ffn, lrow, lval, cnt, a.part, a.pstride, red, pol, a.stamps + 4,
+  stream_rows<BF16, VB, UB, (VB <= 2)>(wt, ffn, lrow, [&](int j) { return load_elem(a.x, a.xdt, j); }, cnt, a.part,
+                                       a.pstride, red, pol, a.stamps + 4,
                             a.cta_t + b * 4 + 1);
   dstamp(a.stamps, 5);
   // this CTA's columns of h: float4 columns [qc0, qc0 + nqc); their down-gate norms are
@@ -477,7 +496,6 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   }
   __syncthreads();
   cnt = list_rows(flags, ffn, G, b, wpre, lrow, a.list_cap, a.status);
-  for (int r = t; r < cnt; r += kDT) lval[r] = __ldcg(a.h + lrow[r]);
   if (b == G - 1)
     for (int j = t; j < ffn; j += kDT) a.keep_d[j] = (uint8_t)((flags[j >> 5] >> (j & 31)) & 1u);
   __syncthreads();
@@ -485,7 +503,8 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   dcta_time(a.cta_t, 2);
 
   // ---------------- E: stream the down rows into this CTA's partial row of y ----------------
-  stream_rows<BF16, VE, UE>(a.wt_down, d, lrow, lval, cnt, a.part, a.pstride, red, pol, a.stamps + 12,
+  stream_rows<BF16, VE, UE, (VE <= 2)>(a.wt_down, d, lrow, [&](int j) { return __ldcg(a.h + j); }, cnt, a.part,
+                                       a.pstride, red, pol, a.stamps + 12,
                             a.cta_t + b * 4 + 3);
   dstamp(a.stamps, 13);
   if (!grid_sync_fixed(a.bar, G, a.status, a.wait_ns)) return;
@@ -506,7 +525,9 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
 // at 1024 threads)
 template <int VPT>
 struct RowsInFlight {
-  static constexpr int value = VPT == 1 ? 8 : (VPT == 2 ? 4 : (VPT == 3 ? 2 : 1));
+  // rows per batch: two register buffers of this many rows for 1 or 2 vectors per thread,
+  // one buffer beyond (the 64 registers of a 1024-thread CTA)
+  static constexpr int value = VPT == 1 ? 4 : (VPT == 2 ? 2 : (VPT == 3 ? 2 : 1));
 };
 
 template <bool BF16, int VB, int VE, int KA, int KC>
@@ -589,7 +610,6 @@ wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int
   p.sm_flags = SL.flags;
   p.sm_wpre = SL.wpre;
   p.sm_lrow = SL.lrow;
-  p.sm_lval = SL.lval;
   p.bar = reinterpret_cast<GridBarrier*>(w + L.bar);
   p.wait_ns = wait_limit_ns();
   p.part = reinterpret_cast<float*>(w + L.part);
