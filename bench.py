@@ -9,13 +9,15 @@ so every step streams its kept rows from HBM.
 Printed (rank 0, one JSON line): effective HBM GB/s on the bytes the kept rows and the
 vectors require (value; whole job), us per layer, the roofline of the fused kernel
 against the measured HBM copy bandwidth (with the ncu DRAM traffic of one launch when
-profiles/ holds it for this kernel source), the dense comparator (the same kernel with
-every channel kept), 16 tokens per call on the batched path (against the union of the
-kept rows), the end-to-end figure through the C ABI with host buffers, and the CPU
-oracle's time on a bounded sample.
+profiles/ holds it for this kernel source), the dense comparator (a dedicated dense
+FFN kernel on the output-major weights), 16 tokens per call on the batched path (against
+the union of the kept rows), the other workloads of the scope table, the end-to-end
+figure through the C ABI with host buffers, and the CPU oracle's time on a bounded
+sample.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--p 0.5] [--layers 8]
   python bench.py --impl reference ...   # the CPU oracle, timed on the host cores
+  python bench.py --profile-case NAME    # one call of a workload three times, for ncu
 """
 
 from __future__ import annotations
@@ -451,6 +453,84 @@ def reduce_max(v: float, world: int, device: str) -> float:
 
 
 
+PROFILE_CASES = ("ffn_decode", "dense_ffn", "union_b256", "batched_b16", "spark_ffn", "ds_decode")
+
+
+def profile_case(name: str) -> None:
+    """One hot-path call of the named workload, three times on one input (the weights once
+    on the device, a few hundred MB), for single-kernel ncu captures: no timing, no
+    output besides a status line. ffn_decode: the Llama-7B FFN at 50% sparsity, bs1 (the
+    single-token kernel); dense_ffn: its dense comparator; union_b256: the ultra-sparse
+    down projection, 256 tokens (the tcgen05 union product); batched_b16: the Llama-7B
+    FFN at 16 tokens; spark_ffn: the Gemma-2-2B FFN with the Spark gate, bs1; ds_decode:
+    Double Sparsity decode attention, Llama-2-7B shapes, 8 sequences."""
+    import torch
+    import free_activation_sparse_b200 as W
+
+    torch.cuda.set_device(0)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if name in ("ffn_decode", "dense_ffn", "batched_b16"):
+        cfg = synth.make_llama7b_ffn(batch=16 if name == "batched_b16" else 1)
+        Wg, Wu, Wd = (_dev_bf16(torch, cfg[k]) for k in ("Wg", "Wu", "Wd"))
+        x = _dev_bf16(torch, cfg["x"])
+        if name == "dense_ffn":
+            ws = W.Workspace(W.OP_DENSE_FFN, D, FFN, 0, 1)
+            calls = [lambda: W.dense_ffn_swiglu(Wg, Wu, Wd, x[0], ws=ws, status=st)]
+        else:
+            f = W.ffn_prepare(Wg, Wu, Wd)
+            del Wg, Wu, Wd
+            B = x.shape[0]
+            ws = W.Workspace(W.OP_FFN_SWIGLU, D, FFN, 0, B)
+            calls = [lambda: W.sparse_ffn_swiglu(f, x, W.GATE_TOPK, cfg["k_gate"], cfg["k_up"], cfg["k_down"], ws=ws,
+                                                 status=st)]
+    elif name == "union_b256":
+        cfg = synth.make_ultrasparse_down()
+        Wt = W.pack_in_major(_dev_bf16(torch, cfg["W"]))
+        xb = _dev_bf16(torch, cfg["x"])
+        idx, xs = W.select_topk(xb, None, cfg["nnz"])
+        ws = W.Workspace(W.OP_SPARSE_MATVEC, cfg["n"], cfg["m"], cfg["nnz"], xb.shape[0])
+        calls = [lambda: W.sparse_matvec(Wt, idx, xs, ws=ws, status=st)]
+    elif name == "spark_ffn":
+        cfg = synth.make_gemma2_2b_spark(batch=1)
+        f = W.ffn_prepare(*(_dev_bf16(torch, cfg[k]) for k in ("Wg", "Wu", "Wd")))
+        x = _dev_bf16(torch, cfg["x_bf16"][:1])
+        ws = W.Workspace(W.OP_FFN_SWIGLU, cfg["d"], cfg["ffn"], 0, 1)
+        calls = [lambda: W.sparse_ffn_swiglu(f, x, W.GATE_STAT, s=cfg["s"], ws=ws, status=st)]
+    elif name == "ds_decode":
+        cfg = synth.make_ds_decode(batch=8)
+        q, K, V = (_dev_bf16(torch, cfg[n]) for n in ("q", "K", "V"))
+        seq = torch.from_numpy(cfg["seq_len"]).cuda()
+        C = torch.from_numpy(cfg["outliers"]).cuda()
+        lab = W.ds_label_build(K, seq, C)
+        calls = [lambda: W.ds_decode_attention(q, K, V, lab, C, seq, 256, status=st)]
+    else:
+        raise SystemExit(f"unknown profile case {name}; one of {PROFILE_CASES}")
+    for _ in range(3):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise SystemExit(f"{name}: device status {int(st.item())}")
+    print(f"ok {name}", flush=True)
+    if name == "ffn_decode":
+        # the single-token kernel's phase stamps (CTA 0's clock at each phase boundary, read
+        # back from the workspace) over 20 more calls, median microseconds per phase
+        phases = ["A keys", "A select", "A flags+list", "B loop", "B store", "barrier 1", "C1 sum",
+                  "barrier 2", "C2 keys", "C2 select", "C2 flags+list", "E loop", "E store", "barrier 3", "E2 sum"]
+        mhz = 1965.0  # SM clock under load in the bench's clock samples (the B200's maximum)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        runs = []
+        for _ in range(20):
+            flush.zero_()
+            calls[0]()
+            torch.cuda.synchronize()
+            sv = W.ffn_ws_view(ws, D, FFN, 1)["stamps"].cpu().numpy()[:16].astype(np.float64)
+            runs.append(np.diff(sv) / mhz)
+        med = np.median(np.array(runs), axis=0)
+        print("phases_us " + json.dumps({n: round(float(v), 2) for n, v in zip(phases, med)}) +
+              f" total {float(med.sum()):.1f} (clock {mhz:.0f} MHz)", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -460,7 +540,12 @@ def main():
     ap.add_argument("--p", type=float, default=0.5, help="dropped fraction per projection")
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
+                    help="run one hot-path call of this workload three times (for ncu) and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     rank = int(os.environ.get("RANK", "0"))
@@ -719,7 +804,7 @@ def main():
 
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
     traffic = None  # ncu dram bytes of one launch, valid only for the kernel it was taken on
-    tf = os.path.join(ROOT, "profiles", "ffn_fused_llama7b_traffic.txt")
+    tf = os.path.join(ROOT, "profiles", "ffn_decode_llama7b_traffic.txt")
     if os.path.exists(tf):
         with open(tf) as f:
             tj = dict(line.strip().split("=", 1) for line in f if "=" in line)
