@@ -8,7 +8,6 @@
 // registers and writes one partial row. When P > 1 the launch is cooperative: after a
 // grid barrier (bounded wait) every CTA sums a slice of the outputs over the P partials
 // in a fixed order, so results are bit-reproducible. When P == 1 the CTA writes y.
-#include <mutex>
 
 #include "internal.h"
 
@@ -214,24 +213,14 @@ constexpr int64_t kNoAllocMaxOutputs = kNoAllocPartialFloats / 2;  // batch * m 
 // [GridBarrier (256 B)][partials: kNoAllocPartialFloats float32]
 static __device__ __align__(256) unsigned char g_noalloc_scratch[256 + kNoAllocPartialFloats * 4];
 
-namespace {
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {nullptr};
-}  // namespace
-
-// Device address of g_noalloc_scratch on the current device. In host code the array's
-// name is only a host-side stand-in, so the address is looked up once per device
-// (with that device current) and cached. Returns nullptr on error.
+// Device address of g_noalloc_scratch in the current context. In host code the array's
+// name is only a host-side stand-in, so the address is looked up on every call (a cheap
+// runtime query), which stays right across a device reset or a new primary context.
+// Returns nullptr on error.
 static void* noalloc_scratch_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_ptr[dev] = p;
-  }
-  return g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace wina
