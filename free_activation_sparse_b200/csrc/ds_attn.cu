@@ -36,43 +36,40 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// n consecutive elements (n = 1, 2, 4 or 8) of a row, starting n-element aligned, widened
-__device__ __forceinline__ void load_lane(const void* p, int dt, int64_t off, int n, float (&out)[8]) {
-  if (dt == WINA_BF16) {
-    const uint16_t* s = reinterpret_cast<const uint16_t*>(p) + off;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (n == 8) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(s));
-      w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
-    } else if (n == 4) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(s));
-      w[0] = v.x, w[1] = v.y;
-    } else if (n == 2) {
+// EPL consecutive elements of one row held as raw words (loaded now, widened when used), so
+// that many rows' loads can be in flight at once.
+template <bool BF16, int EPL>
+struct Lane {
+  static constexpr int BYTES = EPL * (BF16 ? 2 : 4);
+  static constexpr int W = BYTES < 4 ? 1 : BYTES / 4;
+  uint32_t w[W];
+  // elements [off, off + EPL) of p (EPL-element aligned)
+  __device__ __forceinline__ void load(const void* p, int64_t off) {
+    const char* s = reinterpret_cast<const char*>(p) + off * (BF16 ? 2 : 4);
+    if constexpr (BYTES == 2) {
+      w[0] = __ldg(reinterpret_cast<const uint16_t*>(s));
+    } else if constexpr (BYTES == 4) {
       w[0] = __ldg(reinterpret_cast<const uint32_t*>(s));
+    } else if constexpr (BYTES == 8) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(s));
+      w[0] = v.x;
+      w[1] = v.y;
     } else {
-      w[0] = __ldg(s);
-    }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      out[2 * q] = __uint_as_float(w[q] << 16);
-      out[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
-    }
-  } else {
-    const float* s = reinterpret_cast<const float*>(p) + off;
-    if (n >= 4) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(s));
-      out[0] = a.x, out[1] = a.y, out[2] = a.z, out[3] = a.w;
-      if (n == 8) {
-        const float4 b = __ldg(reinterpret_cast<const float4*>(s) + 1);
-        out[4] = b.x, out[5] = b.y, out[6] = b.z, out[7] = b.w;
+      for (int q = 0; q < BYTES / 16; ++q) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(s) + q);
+        w[4 * q] = v.x;
+        w[4 * q + 1] = v.y;
+        w[4 * q + 2] = v.z;
+        w[4 * q + 3] = v.w;
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 2; ++e)
-        if (e < n) out[e] = __ldg(s + e);
     }
   }
-}
+  __device__ __forceinline__ float get(int e) const {
+    if constexpr (BF16) return __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+    else return __uint_as_float(w[e]);
+  }
+};
 
 struct DsParams {
   const void* q;
@@ -92,8 +89,12 @@ struct DsParams {
 };
 
 // Dynamic shared memory: keys [Tmax] | sel [kcap] | logits [kcap] | hist [kSelBins] |
-// cand [2 kSelCand] | q [dh] | part [kAW][dh]
+// cand [2 kSelCand] | q [dh] | part [kAW][dh]. EPL = dh / 32 channels per lane.
+template <bool BF16, int EPL>
 __global__ void __launch_bounds__(kAT, 1) k_ds_decode(DsParams p) {
+  constexpr int LV = BF16 ? 8 : 4;                    // label elements per 16-byte piece
+  constexpr int TPT = 8;                              // tokens a thread scores per pass
+  constexpr int SPW = Lane<BF16, EPL>::W >= 8 ? 4 : (Lane<BF16, EPL>::W >= 4 ? 8 : 16);  // kept tokens per warp per pass
   extern __shared__ __align__(16) uint32_t dsm[];
   const int kcap = min(p.k, p.Tmax);
   uint32_t* keys = dsm;
@@ -123,20 +124,34 @@ __global__ void __launch_bounds__(kAT, 1) k_ds_decode(DsParams p) {
   for (int j = tid; j < p.r; j += kAT) qc[j] = qf[__ldg(p.channels + (int64_t)g * p.r + j)];
   __syncthreads();
 
-  // step 2: approximate scores against the label rows, as order-preserving keys
-  const int lv = p.kvdt == WINA_BF16 ? 8 : 4;  // label elements per 16-byte load
-  for (int t = tid; t < T; t += kAT) {
-    const int64_t row = (head * p.Tmax + t) * p.r;
-    float s = 0.f;
-    for (int j0 = 0; j0 < p.r; j0 += lv) {
-      float l[8];
-      load_lane(p.label, p.kvdt, row + j0, lv, l);
+  // step 2: approximate scores against the label rows, as order-preserving keys. A thread
+  // takes tokens tid + u * kAT (u < TPT) per pass; each 16-byte piece of their label rows
+  // is loaded for all of them at once, and every token's products are summed in channel
+  // order.
+  for (int t0 = tid; t0 < T; t0 += kAT * TPT) {
+    float s[TPT];
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (e < lv) s = __fadd_rn(s, __fmul_rn(qc[j0 + e], l[e]));  // channel order
+    for (int u = 0; u < TPT; ++u) s[u] = 0.f;
+    for (int j0 = 0; j0 < p.r; j0 += LV) {
+      Lane<BF16, LV> lab[TPT];
+#pragma unroll
+      for (int u = 0; u < TPT; ++u)
+        if (t0 + u * kAT < T) lab[u].load(p.label, (head * p.Tmax + t0 + u * kAT) * p.r + j0);
+#pragma unroll
+      for (int u = 0; u < TPT; ++u)
+        if (t0 + u * kAT < T) {
+#pragma unroll
+          for (int e = 0; e < LV; ++e) s[u] = __fadd_rn(s[u], __fmul_rn(qc[j0 + e], lab[u].get(e)));
+        }
     }
-    keys[t] = order_key(s);
-    if (p.scores_out) p.scores_out[((int64_t)b * p.Hq + h) * p.Tmax + t] = s;
+#pragma unroll
+    for (int u = 0; u < TPT; ++u) {
+      const int t = t0 + u * kAT;
+      if (t < T) {
+        keys[t] = order_key(s[u]);
+        if (p.scores_out) p.scores_out[((int64_t)b * p.Hq + h) * p.Tmax + t] = s[u];
+      }
+    }
   }
   __syncthreads();
 
@@ -157,69 +172,136 @@ __global__ void __launch_bounds__(kAT, 1) k_ds_decode(DsParams p) {
   if (p.idx_out)
     for (int i = tid; i < kk; i += kAT) p.idx_out[((int64_t)b * p.Hq + h) * p.k + i] = sel[i];
 
-  // attention over the kept tokens: logits, one warp per token (lanes over channels)
-  const int epl = p.dh / 32;  // channels per lane (dh is a multiple of 32)
-  for (int i = warp; i < kk; i += kAW) {
-    const int64_t row = (head * p.Tmax + sel[i]) * p.dh + (int64_t)lane * epl;
-    float kv[8];
-    load_lane(p.K, p.kvdt, row, epl, kv);
-    float dot = 0.f;
+  // attention over the kept tokens. Warp w takes kept tokens w + u * kAW (u < SPW) per
+  // pass, lanes over channels; their key and value pieces are loaded together, the
+  // logits go to SMEM, and the value pieces wait in registers for the softmax weights.
+  float acc[EPL];
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (e < epl) dot = fmaf(qf[lane * epl + e], kv[e], dot);
+  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+  const int npass = (kk + kAW * SPW - 1) / (kAW * SPW);
+  float mx = -INFINITY, sum = 0.f;
+  for (int ps = 0; ps < npass; ++ps) {
+    const int i0 = ps * kAW * SPW + warp;
+    Lane<BF16, EPL> kr[SPW], vr[SPW];
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (lane == 0) logits[i] = dot * p.scale;
+    for (int u = 0; u < SPW; ++u) {
+      const int i = i0 + u * kAW;
+      if (i < kk) {
+        const int64_t row = (head * p.Tmax + sel[i]) * p.dh + (int64_t)lane * EPL;
+        kr[u].load(p.K, row);
+        vr[u].load(p.V, row);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < SPW; ++u) {
+      const int i = i0 + u * kAW;
+      if (i < kk) {  // warp-uniform
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) dot = fmaf(qf[lane * EPL + e], kr[u].get(e), dot);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (lane == 0) logits[i] = dot * p.scale;
+      }
+    }
+    // the softmax needs every logit: with one pass (kk <= kAW * SPW) the value pieces stay
+    // in registers across it; with several, the max and sum come after the last pass and
+    // the weighted values are added in a second sweep below
+    if (npass == 1) {
+      __syncthreads();
+      for (int i = tid; i < kk; i += kAT) mx = fmaxf(mx, logits[i]);
+      {
+        float m = mx;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) fred[warp] = m;
+        __syncthreads();
+        m = fred[0];
+        for (int w = 1; w < kAW; ++w) m = fmaxf(m, fred[w]);
+        __syncthreads();
+        mx = m;
+      }
+      for (int i = tid; i < kk; i += kAT) {
+        const float e = expf(logits[i] - mx);
+        logits[i] = e;
+        sum += e;
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0) fred[warp] = sum;
+      __syncthreads();
+      {
+        float s2 = 0.f;
+        for (int w = 0; w < kAW; ++w) s2 += fred[w];
+        sum = s2;
+      }
+#pragma unroll
+      for (int u = 0; u < SPW; ++u) {
+        const int i = i0 + u * kAW;
+        if (i < kk) {
+          const float wgt = logits[i];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) acc[e] = fmaf(wgt, vr[u].get(e), acc[e]);
+        }
+      }
+    }
   }
-  __syncthreads();
-  float mx = -INFINITY;
-  for (int i = tid; i < kk; i += kAT) mx = fmaxf(mx, logits[i]);
-  {
-    float m = mx;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) fred[warp] = m;
+  if (npass > 1) {
+    // several passes: softmax over all logits, then the weighted value rows again in
+    // batches (their loads issued together per pass)
     __syncthreads();
-    m = fred[0];
-    for (int w = 1; w < kAW; ++w) m = fmaxf(m, fred[w]);
-    __syncthreads();
-    mx = m;
-  }
-  float sum = 0.f;
-  for (int i = tid; i < kk; i += kAT) {
-    const float e = expf(logits[i] - mx);
-    logits[i] = e;
-    sum += e;
-  }
-  {
+    for (int i = tid; i < kk; i += kAT) mx = fmaxf(mx, logits[i]);
+    {
+      float m = mx;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) fred[warp] = m;
+      __syncthreads();
+      m = fred[0];
+      for (int w = 1; w < kAW; ++w) m = fmaxf(m, fred[w]);
+      __syncthreads();
+      mx = m;
+    }
+    for (int i = tid; i < kk; i += kAT) {
+      const float e = expf(logits[i] - mx);
+      logits[i] = e;
+      sum += e;
+    }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (lane == 0) fred[warp] = sum;
     __syncthreads();
-    float s = 0.f;
-    for (int w = 0; w < kAW; ++w) s += fred[w];
-    sum = s;
+    {
+      float s2 = 0.f;
+      for (int w = 0; w < kAW; ++w) s2 += fred[w];
+      sum = s2;
+    }
+    for (int ps = 0; ps < npass; ++ps) {
+      const int i0 = ps * kAW * SPW + warp;
+      Lane<BF16, EPL> vr[SPW];
+#pragma unroll
+      for (int u = 0; u < SPW; ++u) {
+        const int i = i0 + u * kAW;
+        if (i < kk) vr[u].load(p.V, (head * p.Tmax + sel[i]) * p.dh + (int64_t)lane * EPL);
+      }
+#pragma unroll
+      for (int u = 0; u < SPW; ++u) {
+        const int i = i0 + u * kAW;
+        if (i < kk) {
+          const float wgt = logits[i];
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) acc[e] = fmaf(wgt, vr[u].get(e), acc[e]);
+        }
+      }
+    }
   }
-  // weighted value rows: warp w takes the kept tokens i = w, w + 16, ...
-  float acc[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int i = warp; i < kk; i += kAW) {
-    float v[8];
-    load_lane(p.V, p.kvdt, (head * p.Tmax + sel[i]) * p.dh + (int64_t)lane * epl, epl, v);
-    const float w = logits[i];
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (e < epl) acc[e] = fmaf(w, v[e], acc[e]);
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-    if (e < epl) part[warp * p.dh + lane * epl + e] = acc[e];
+  for (int e = 0; e < EPL; ++e) part[warp * p.dh + lane * EPL + e] = acc[e];
   __syncthreads();
   for (int d = tid; d < p.dh; d += kAT) {
-    float s = 0.f;
-    for (int w = 0; w < kAW; ++w) s += part[w * p.dh + d];
-    out[d] = s / sum;
+    float s2 = 0.f;
+    for (int w = 0; w < kAW; ++w) s2 += part[w * p.dh + d];
+    out[d] = s2 / sum;
   }
 }
 
@@ -346,11 +428,19 @@ extern "C" wina_status_t ds_decode_attention(const void* q, wina_dtype_t qdt, co
   p.status = status_dev;
   const size_t smem = ds_decode_smem_bytes(Tmax, dh, k);
   if (smem > kDsMaxSmem) return WINA_ERR_INVALID_ARG;  // Tmax and min(k, Tmax) too large together
+  void (*kern)(DsParams) = nullptr;
+  const bool bf = kvdt == WINA_BF16;
+  switch (dh) {
+    case 32: kern = bf ? k_ds_decode<true, 1> : k_ds_decode<false, 1>; break;
+    case 64: kern = bf ? k_ds_decode<true, 2> : k_ds_decode<false, 2>; break;
+    case 128: kern = bf ? k_ds_decode<true, 4> : k_ds_decode<false, 4>; break;
+    default: kern = bf ? k_ds_decode<true, 8> : k_ds_decode<false, 8>; break;
+  }
   {
     // always: the kernel's static shared memory comes on top of the dynamic part
-    const cudaError_t e = ensure_smem_limit((const void*)k_ds_decode, smem);
+    const cudaError_t e = ensure_smem_limit((const void*)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
   }
-  k_ds_decode<<<(unsigned)(B * Hq), kAT, smem, (cudaStream_t)stream>>>(p);
+  kern<<<(unsigned)(B * Hq), kAT, smem, (cudaStream_t)stream>>>(p);
   return cuda_status(cudaGetLastError());
 }
