@@ -200,7 +200,7 @@ __device__ int list_rows(const uint32_t* flags, int n, int parts, int part, uint
 // streaming the listed rows
 // ------------------------------------------------------------------------------------
 
-// This CTA's partial row(s) of sum over the listed rows r of val(lrow[r]) *
+// This CTA's partial row(s) of sum over the listed rows r of val(lrow[r], r) *
 // Wt[lrow[r]][0..m), read with 16-byte loads, stored in `part` (row stride pstride floats).
 // The CTA is split into NG = kDT / TPR groups of TPR threads; group g takes list entries
 // g, g + NG, ...; thread l of a group owns VPT vectors of each row, those of index l,
@@ -243,7 +243,7 @@ __device__ void stream_rows(const void* __restrict__ Wt, int m, const int* lrow,
     for (int u = 0; u < U; ++u) {
       if (i0 + u < mine) {
         const int row = lrow[g + (i0 + u) * NG];
-        xv[u] = val(row);
+        xv[u] = val(row, g + (i0 + u) * NG);
         const uint4* rp = base + (int64_t)row * V;
 #pragma unroll
         for (int j = 0; j < VPT; ++j)
@@ -436,9 +436,8 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   dcta_time(a.cta_t, 0);
 
   // ---------------- B: stream the gate / up rows into this CTA's partial row ----------------
-  stream_rows<BF16, VB, UB, (VB <= 2)>(wt, ffn, lrow, [&](int j) { return load_elem(a.x, a.xdt, j); }, cnt, a.part,
-                                       a.pstride, red, pol, a.stamps + 4,
-                            a.cta_t + b * 4 + 1);
+  stream_rows<BF16, VB, UB, (VB <= 2)>(wt, ffn, lrow, [&](int j, int) { return load_elem(a.x, a.xdt, j); }, cnt,
+                                       a.part, a.pstride, red, pol, a.stamps + 4, a.cta_t + b * 4 + 1);
   dstamp(a.stamps, 5);
   // this CTA's columns of h: float4 columns [qc0, qc0 + nqc); their down-gate norms are
   // read now and used after the barrier
@@ -453,7 +452,8 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   touch_pages_d(a.wt_down, (size_t)d * ffn * ESZ);
   {
     float4 g4, u4;
-    reduce_scatter(a.part, a.pstride, qc0, nqc, a.Gg * npb, G * npb, reinterpret_cast<float4*>(red), &g4, &u4);
+    reduce_scatter(a.part, a.pstride, qc0, nqc, a.Gg * npb, G * npb, reinterpret_cast<float4*>(red), &g4,
+                             &u4);
     if (t < nqc) {
       const int q = qc0 + t;
       const float4 h4 = make_float4(silu_d(g4.x) * u4.x, silu_d(g4.y) * u4.y, silu_d(g4.z) * u4.z,
@@ -503,9 +503,8 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
   dcta_time(a.cta_t, 2);
 
   // ---------------- E: stream the down rows into this CTA's partial row of y ----------------
-  stream_rows<BF16, VE, UE, (VE <= 2)>(a.wt_down, d, lrow, [&](int j) { return __ldcg(a.h + j); }, cnt, a.part,
-                                       a.pstride, red, pol, a.stamps + 12,
-                            a.cta_t + b * 4 + 3);
+  stream_rows<BF16, VE, UE, (VE <= 2)>(a.wt_down, d, lrow, [&](int j, int) { return __ldcg(a.h + j); }, cnt, a.part,
+                                       a.pstride, red, pol, a.stamps + 12, a.cta_t + b * 4 + 3);
   dstamp(a.stamps, 13);
   if (!grid_sync_fixed(a.bar, G, a.status, a.wait_ns)) return;
   dstamp(a.stamps, 14);
@@ -515,7 +514,8 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
     const int q0 = (int)((int64_t)(d / 4) * b / G);
     const int nq = (int)((int64_t)(d / 4) * (b + 1) / G) - q0;
     float4 y4, unused;
-    reduce_scatter(a.part, a.pstride, q0, nq, G * npe, G * npe, reinterpret_cast<float4*>(red), &y4, &unused);
+    reduce_scatter(a.part, a.pstride, q0, nq, G * npe, G * npe, reinterpret_cast<float4*>(red), &y4,
+                             &unused);
     if (t < nq) reinterpret_cast<float4*>(a.y)[q0 + t] = y4;
   }
   dstamp(a.stamps, 15);
@@ -642,6 +642,149 @@ wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int
   }
   void* args[] = {&p};
   return cuda_status(cudaLaunchKernelExC(&cfg, kern, args));
+}
+
+// ------------------------------------------------------------------------------------
+// one token's sparse product on the same row stream
+// ------------------------------------------------------------------------------------
+//
+// y[:] = sum over r < k of xs[r] * Wt[idx[r]][:] ("Spark Transformer", section 3.1, SVMM)
+// for a single token: one cooperative launch of one 1024-thread CTA per SM. CTA c takes
+// list entries c, c + G, c + 2G, ... (the kept rows dealt out round robin, so that all SMs
+// read rows from the same neighbourhood of the weight at any moment), streams them as the
+// FFN kernel's phase B does and stores its partial rows; after a grid barrier CTA c sums
+// its slice of the columns over all partial rows in a fixed order. Bit-reproducible.
+
+struct SpmvOneParams {
+  const void* Wt;
+  int64_t n;
+  int m;
+  const int32_t* idx;
+  const float* xs;
+  int k_fixed;            // >= 0: entries of the list; -1: count[0], clamped to ld
+  const int32_t* count;
+  int ld;
+  float* y;
+  float* part;            // [2G][m + 4] float32 partial rows
+  GridBarrier* bar;
+  int cap;                // list entries per CTA at most
+  unsigned long long wait_ns;
+  int32_t* status;
+};
+
+template <bool BF16, int VPT>
+__global__ void __launch_bounds__(kDT, 1) k_spmv_one(SpmvOneParams a) {
+  constexpr int U = RowsInFlight<VPT>::value;
+  extern __shared__ __align__(128) unsigned char smraw[];
+  int* lrow = reinterpret_cast<int*>(smraw);            // [cap]
+  float* lval = reinterpret_cast<float*>(lrow + a.cap);  // [cap]
+  float* red = lval + a.cap;                             // reduction scratch (16-byte aligned: cap % 4 == 0)
+  const int G = gridDim.x, c = blockIdx.x, t = threadIdx.x;
+  const uint64_t pol = l2_evict_first_policy();
+  int kb = a.k_fixed;
+  if (kb < 0) kb = max(0, min(__ldg(a.count), a.ld));
+  int cnt = kb > c ? (kb - c + G - 1) / G : 0;
+  if (cnt > a.cap) {  // cannot happen with the launcher's cap; kept as a guard
+    if (t == 0) record_status(a.status, WINA_ERR_CAPACITY);
+    cnt = a.cap;
+  }
+  for (int i = t; i < cnt; i += kDT) {
+    const int r = c + i * G;
+    int32_t row = __ldg(a.idx + r);
+    float v = __ldg(a.xs + r);
+    if (row < 0 || (int64_t)row >= a.n) {  // never read outside Wt
+      record_status(a.status, WINA_ERR_INVALID_ARG);
+      row = 0;
+      v = 0.f;
+    }
+    lrow[i] = row;
+    lval[i] = v;
+  }
+  __syncthreads();
+  unsigned long long unused_t;
+  long long unused_s;
+  const int pstride = a.m + 4;  // rows offset by 4 floats: one column of successive rows spreads over L2 slices
+  stream_rows<BF16, VPT, U, (VPT <= 2)>(a.Wt, a.m, lrow, [&](int, int pos) { return lval[pos]; }, cnt, a.part,
+                                        pstride, red, pol, &unused_s, &unused_t);
+  if (!grid_sync_fixed(a.bar, G, a.status, a.wait_ns)) return;
+  constexpr uint32_t ESZ = BF16 ? 2u : 4u;
+  const int np = decode_partials(a.m * (int)ESZ / 16);
+  const int q0 = (int)((int64_t)(a.m / 4) * c / G);
+  const int nq = (int)((int64_t)(a.m / 4) * (c + 1) / G) - q0;
+  float4 y4, unused;
+  reduce_scatter(a.part, pstride, q0, nq, G * np, G * np, reinterpret_cast<float4*>(red), &y4, &unused);
+  if (t < nq) reinterpret_cast<float4*>(a.y)[q0 + t] = y4;
+}
+
+template <bool BF16, int VPT>
+static wina_status_t launch_spmv_one_t(SpmvOneParams p, int G, cudaStream_t st) {
+  void* kern = (void*)k_spmv_one<BF16, VPT>;
+  const int esz = BF16 ? 2 : 4;
+  const int V = p.m * esz / 16;
+  const int tpr = decode_tpr(V);
+  const int red_floats = std::max((kDT / tpr - 1) * tpr * (16 / esz), 32 * 32 * 4);
+  const size_t smem = (size_t)p.cap * 8 + (size_t)red_floats * 4;
+  cudaError_t e = ensure_smem_limit(kern, smem);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = ensure_prefer_l1(kern);  // the weight loads in flight live in L1
+  if (e != cudaSuccess) return cuda_status(e);
+  if (blocks_per_sm(kern, kDT, smem) < 1) return WINA_ERR_UNSUPPORTED_DTYPE;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)G);
+  cfg.blockDim = dim3(kDT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[] = {&p};
+  return cuda_status(cudaLaunchKernelExC(&cfg, kern, args));
+}
+
+wina_status_t launch_spmv_one(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx, const float* xs,
+                              int k, const int32_t* count, int ld, float* y, float* part, GridBarrier* bar,
+                              int32_t* status, cudaStream_t st) {
+  const bool bf16 = wdt == WINA_BF16;
+  const int esz = bf16 ? 2 : 4;
+  const int vpt = decode_vpt(m, esz);
+  const int sms = device_sm_count();
+  const int G = std::min(sms, kGridCap / 2);  // 2G partial rows fit the workspace's kGridCap
+  if (vpt == 0 || G < 2 || m > INT32_MAX) return WINA_ERR_UNSUPPORTED_DTYPE;
+  if ((m / 4 + G - 1) / G > 32) return WINA_ERR_UNSUPPORTED_DTYPE;  // one lane per float4 column
+  const int kmax = k >= 0 ? k : ld;
+  SpmvOneParams p;
+  p.Wt = Wt;
+  p.n = n;
+  p.m = (int)m;
+  p.idx = idx;
+  p.xs = xs;
+  p.k_fixed = k;
+  p.count = count;
+  p.ld = ld;
+  p.y = y;
+  p.part = part;
+  p.bar = bar;
+  p.cap = ((kmax + G - 1) / G + 3) / 4 * 4;
+  if (p.cap < 4) p.cap = 4;
+  p.wait_ns = wait_limit_ns();
+  p.status = status;
+  if ((size_t)p.cap * 8 > 64 * 1024) return WINA_ERR_UNSUPPORTED_DTYPE;  // list beyond SMEM: the general path
+  if (bf16) {
+    switch (vpt) {
+      case 1: return launch_spmv_one_t<true, 1>(p, G, st);
+      case 2: return launch_spmv_one_t<true, 2>(p, G, st);
+      case 3: return launch_spmv_one_t<true, 3>(p, G, st);
+      default: return launch_spmv_one_t<true, 4>(p, G, st);
+    }
+  }
+  switch (vpt) {
+    case 1: return launch_spmv_one_t<false, 1>(p, G, st);
+    case 2: return launch_spmv_one_t<false, 2>(p, G, st);
+    case 3: return launch_spmv_one_t<false, 3>(p, G, st);
+    default: return launch_spmv_one_t<false, 4>(p, G, st);
+  }
 }
 
 }  // namespace wina

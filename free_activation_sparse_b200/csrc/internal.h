@@ -83,8 +83,8 @@ int max_coresident_grid(K kern, int threads, size_t smem) {
 // workspace layouts
 // ----------------------------------------------------------------------------------
 
-// sparse_matvec: [GridBarrier][partials: kGridCap x m float32]. Only needed when a
-// token is split over several CTAs (batch < kGridCap).
+// sparse_matvec: [GridBarrier][partials: kGridCap x (m + 4) float32]. The partial rows
+// are only needed when a token is split over several CTAs (batch < kGridCap).
 struct SpmvWs {
   size_t bar, partials, total;
 };
@@ -92,7 +92,7 @@ inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
   SpmvWs w;
   w.bar = 0;
   w.partials = kAlign;
-  const size_t part = batch < kGridCap ? (size_t)kGridCap * (size_t)m * 4 : 0;
+  const size_t part = batch < kGridCap ? (size_t)kGridCap * (size_t)(m + 4) * 4 : 0;
   w.total = round_up(w.partials + part, kAlign);
   return w;
 }
@@ -185,6 +185,13 @@ size_t dense_ws_size(int64_t d, int64_t ffn);
 wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const int32_t* idx, const float* xs, int k,
                                   const int32_t* count, int ld, int batch, float* y, void* ws, int32_t* status,
                                   cudaStream_t s);
+// One token's sparse product on the single-token FFN kernel's row stream (ffn_decode.cu):
+// part has room for 2 * min(SMs, kGridCap / 2) rows of m + 4 floats; bar is a grid
+// barrier of the workspace. Returns WINA_ERR_UNSUPPORTED_DTYPE without launching when the
+// shape is outside what it takes.
+wina_status_t launch_spmv_one(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx, const float* xs,
+                              int k, const int32_t* count, int ld, float* y, float* part, GridBarrier* bar,
+                              int32_t* status, cudaStream_t st);
 // The single-token FFN kernel (ffn_decode.cu). Returns WINA_ERR_UNSUPPORTED_DTYPE without
 // launching anything when the shape is outside what it takes.
 wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int mode, int k_gate, int k_up,

@@ -139,6 +139,13 @@ wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m
   if (batch >= kUnionMinBatch && union_path_takes(wdt, n, m, batch))
     return launch_union_matvec(Wt, n, m, idx, xs, k, count, ld_idx, batch, y,
                                (char*)ws + spmv_ws_layout(m, batch).total, status_dev, s);
+  if (batch == 1) {  // one token: the single-token kernel's row stream, when it takes the shape
+    const SpmvWs L1 = spmv_ws_layout(m, 1);
+    const wina_status_t r1 = launch_spmv_one(Wt, wdt, n, m, idx, xs, k, count, ld_idx, y,
+                                             reinterpret_cast<float*>((char*)ws + L1.partials),
+                                             reinterpret_cast<GridBarrier*>((char*)ws + L1.bar), status_dev, s);
+    if (r1 != WINA_ERR_UNSUPPORTED_DTYPE) return r1;
+  }
   const bool bf16 = wdt == WINA_BF16;
   const size_t smem = spmv_smem();
   const int gmax = bf16 ? max_coresident_grid(k_sparse_matvec<true>, kNT, smem)
