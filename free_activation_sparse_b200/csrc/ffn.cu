@@ -5,38 +5,14 @@
 //
 // The C-ABI entry point. One token takes the single persistent kernel of ffn_decode.cu;
 // several tokens (or shapes that kernel does not take) run as a sequence of batched
-// calls: the gates of gate and up, their sparse products, silu(g) * u, the down gate and
-// the down product.
+// calls: per projection its gate (which also writes the kept-set bytes and, for the union
+// path, the union's flags) and its sparse product, with silu(g) * u before the down gate.
 #include <math.h>
 
 #include <algorithm>
 #include <cmath>
 
 #include "internal.h"
-
-namespace wina {
-
-// Byte flags of kept channels from index lists (the multi-token path's diagnostic view).
-__global__ void k_keep_bytes(const int32_t* __restrict__ idx, int ld, int k, const int32_t* __restrict__ count, int n,
-                             uint8_t* __restrict__ keep) {
-  const int b = blockIdx.x;
-  uint8_t* row = keep + (int64_t)b * n;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) row[j] = 0;
-  __syncthreads();
-  const int kb = k >= 0 ? k : min(count[b], ld);
-  for (int r = threadIdx.x; r < kb; r += blockDim.x) {
-    const int j = idx[(int64_t)b * ld + r];
-    if (j >= 0 && j < n) row[j] = 1;
-  }
-}
-
-static wina_status_t launch_keep_bytes(const int32_t* idx, int ld, int k, const int32_t* count, int n, int B,
-                                       uint8_t* keep, cudaStream_t s) {
-  k_keep_bytes<<<B, 256, 0, s>>>(idx, ld, k, count, n, keep);
-  return cuda_status(cudaGetLastError());
-}
-
-}  // namespace wina
 
 using namespace wina;
 
@@ -94,40 +70,46 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
   float* u = reinterpret_cast<float*>(w + L.u);
   void* sw = w + L.spmv;
   const int B = (int)batch;
+  // union flags of each projection's product (set by the gate that makes its lists, when
+  // the union path serves the call); gate and up share the workspace, so each gate runs
+  // right before its own product
+  uint8_t* uf_gu = union_flags_for(sw, f->wdt, d, ffn, B);
+  uint8_t* uf_d = union_flags_for(sw, f->wdt, ffn, d, B);
   wina_status_t r;
   if (mode == WINA_GATE_STAT) {
     // gate and up threshold the same signed x: one kept set serves both
-    if ((r = launch_stat_threshold(x, xdt, (int)d, z, B, ig, xg, cnt, nullptr, (int)d, status_dev, st))) return r;
-    if ((r = launch_keep_bytes(ig, (int)d, -1, cnt, (int)d, B, keep_g, st))) return r;
+    if ((r = launch_stat_threshold(x, xdt, (int)d, z, B, ig, xg, cnt, nullptr, (int)d, status_dev, st, keep_g, uf_gu)))
+      return r;
     if ((r = cuda_status(cudaMemcpyAsync(keep_u, keep_g, (size_t)B * d, cudaMemcpyDeviceToDevice, st)))) return r;
-    if ((r = launch_sparse_matvec(f->wt_gate, f->wdt, d, ffn, ig, xg, -1, cnt, (int)d, B, g, sw, status_dev, st)))
+    if ((r = launch_sparse_matvec(f->wt_gate, f->wdt, d, ffn, ig, xg, -1, cnt, (int)d, B, g, sw, status_dev, st,
+                                  uf_gu != nullptr)))
       return r;
     if ((r = launch_sparse_matvec(f->wt_up, f->wdt, d, ffn, ig, xg, -1, cnt, (int)d, B, u, sw, status_dev, st)))
       return r;
     if ((r = launch_silu_mul(g, u, h, (int64_t)B * ffn, st))) return r;
     if ((r = launch_stat_threshold(h, WINA_F32, (int)ffn, z, B, idn, xd, cnt + 2 * B, nullptr, (int)ffn, status_dev,
-                                   st)))
+                                   st, keep_d, uf_d)))
       return r;
-    if ((r = launch_keep_bytes(idn, (int)ffn, -1, cnt + 2 * B, (int)ffn, B, keep_d, st))) return r;
     return launch_sparse_matvec(f->wt_down, f->wdt, ffn, d, idn, xd, -1, cnt + 2 * B, (int)ffn, B, y, sw, status_dev,
-                                st);
+                                st, uf_d != nullptr);
   }
   const float* cg = mode == WINA_GATE_TOPK ? f->c_gate : nullptr;
   const float* cu = mode == WINA_GATE_TOPK ? f->c_up : nullptr;
   const float* cd = mode == WINA_GATE_TOPK ? f->c_down : nullptr;
-  if ((r = launch_select_topk(x, xdt, cg, (int)d, (int)k_gate, B, ig, xg, (int)d, nullptr, st))) return r;
-  if ((r = launch_select_topk(x, xdt, cu, (int)d, (int)k_up, B, iu, xu, (int)d, nullptr, st))) return r;
-  if ((r = launch_keep_bytes(ig, (int)d, (int)k_gate, nullptr, (int)d, B, keep_g, st))) return r;
-  if ((r = launch_keep_bytes(iu, (int)d, (int)k_up, nullptr, (int)d, B, keep_u, st))) return r;
+  if ((r = launch_select_topk(x, xdt, cg, (int)d, (int)k_gate, B, ig, xg, (int)d, nullptr, st, keep_g, uf_gu)))
+    return r;
   if ((r = launch_sparse_matvec(f->wt_gate, f->wdt, d, ffn, ig, xg, (int)k_gate, nullptr, (int)d, B, g, sw,
-                                status_dev, st)))
+                                status_dev, st, uf_gu != nullptr)))
+    return r;
+  if ((r = launch_select_topk(x, xdt, cu, (int)d, (int)k_up, B, iu, xu, (int)d, nullptr, st, keep_u, uf_gu)))
     return r;
   if ((r = launch_sparse_matvec(f->wt_up, f->wdt, d, ffn, iu, xu, (int)k_up, nullptr, (int)d, B, u, sw, status_dev,
-                                st)))
+                                st, uf_gu != nullptr)))
     return r;
   if ((r = launch_silu_mul(g, u, h, (int64_t)B * ffn, st))) return r;
-  if ((r = launch_select_topk(h, WINA_F32, cd, (int)ffn, (int)k_down, B, idn, xd, (int)ffn, nullptr, st))) return r;
-  if ((r = launch_keep_bytes(idn, (int)ffn, (int)k_down, nullptr, (int)ffn, B, keep_d, st))) return r;
+  if ((r = launch_select_topk(h, WINA_F32, cd, (int)ffn, (int)k_down, B, idn, xd, (int)ffn, nullptr, st, keep_d,
+                              uf_d)))
+    return r;
   return launch_sparse_matvec(f->wt_down, f->wdt, ffn, d, idn, xd, (int)k_down, nullptr, (int)ffn, B, y, sw,
-                              status_dev, st);
+                              status_dev, st, uf_d != nullptr);
 }

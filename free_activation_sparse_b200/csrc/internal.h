@@ -98,18 +98,19 @@ inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
 }
 
 // The union path of the sparse product (several tokens, bf16 weights): a byte flag per
-// channel [n], per 64-channel block its first X~ column [nblk], the chunk list [nblk + 1],
-// the channel of each gather slot [kmax], each member's X~ column [n], chunk counts and
-// the number of bf16 parts [4], and X~ [3 * np][kmax] bf16 (np = tokens per block rounded
-// up to 16, kmax = 64 * (nblk + 1)).
+// channel [n], the chunk list [nblk + 1], the channel of each gather slot [kmax], each
+// member's X~ column [n], chunk counts and the number of bf16 parts [4], and X~
+// [3 * np][kmax] bf16 (np = tokens per block rounded up to 16, kmax = 64 * (nblk + 1)).
+// The flags and X~ are zero between calls (each call clears what it set).
 struct UnionWs {
-  size_t flag, base, chunk_row, slot, pos, info, xt, total;
+  size_t flag, chunk_row, slot, pos, info, xt, total;
   int64_t kmax, np;
 };
 UnionWs union_ws_layout(int64_t n, int64_t batch);
 // Whether the union path serves this call (bf16 weights, several tokens).
 bool union_path_takes(int wdt, int64_t n, int64_t m, int64_t batch);
 constexpr int kUnionMinBatch = 4;  // fewer tokens take the per-token product
+constexpr int kUnionBlock = 256;   // tokens per union block
 
 // sparse_matvec's workspace: the per-token layout, then the union path's (several tokens)
 inline size_t spmv_total_ws(int64_t n, int64_t m, int64_t batch) {
@@ -170,21 +171,30 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
 // launchers implemented in the kernel files (arguments already checked)
 // ----------------------------------------------------------------------------------
 
+// keep (optional): the kept set as bytes [batch][n]; uflag (optional): the union flags of
+// the union path, set to 1 at every token's kept channels.
 wina_status_t launch_select_topk(const void* x, int xdt, const float* c, int n, int k, int batch, int32_t* idx,
-                                 float* xs, int ld, float* scores, cudaStream_t s);
+                                 float* xs, int ld, float* scores, cudaStream_t s, uint8_t* keep = nullptr,
+                                 uint8_t* uflag = nullptr);
 wina_status_t launch_stat_threshold(const void* v, int vdt, int n, double z, int batch, int32_t* idx, float* xs,
-                                    int32_t* count, float* t, int cap, int32_t* status_dev, cudaStream_t s);
+                                    int32_t* count, float* t, int cap, int32_t* status_dev, cudaStream_t s,
+                                    uint8_t* keep = nullptr, uint8_t* uflag = nullptr);
 wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx,
                                    const float* xs, int k, const int32_t* count, int ld_idx, int batch, float* y,
-                                   void* ws, int32_t* status_dev, cudaStream_t s);
+                                   void* ws, int32_t* status_dev, cudaStream_t s, bool premarked = false);
+// The union flags in sparse_matvec's workspace `ws` for this call, when the union path
+// serves it with a single token block (so that a gate can mark them); nullptr otherwise.
+uint8_t* union_flags_for(void* ws, int wdt, int64_t n, int64_t m, int64_t batch);
 wina_status_t launch_silu_mul(const float* g, const float* u, float* h, int64_t count, cudaStream_t s);
 // Workspace bytes of spark_ffn_swiglu (spark.cu).
 size_t spark_ws_size(int64_t d, int64_t ffn);
 size_t dense_ws_size(int64_t d, int64_t ffn);
-// The union path (union_gemm.cu); ws is the union region of the workspace.
+// The union path (union_gemm.cu); ws is the union region of the workspace. premarked: the
+// union flags were already set by the gate that made the lists (launch_select_topk's
+// uflag), which serves a single token block (batch <= kUBlock).
 wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const int32_t* idx, const float* xs, int k,
                                   const int32_t* count, int ld, int batch, float* y, void* ws, int32_t* status,
-                                  cudaStream_t s);
+                                  cudaStream_t s, bool premarked = false);
 // One token's sparse product on the single-token FFN kernel's row stream (ffn_decode.cu):
 // part has room for 2 * min(SMs, kGridCap / 2) rows of m + 4 floats; bar is a grid
 // barrier of the workspace. Returns WINA_ERR_UNSUPPORTED_DTYPE without launching when the

@@ -17,10 +17,23 @@
 
 namespace wina {
 
+// The kept set as bytes (optional): keep[j] = 1 or 0 for every channel j < n, and the
+// union flags uflag[j] = 1 for the kept channels (several tokens may store the same 1).
+template <int NT, typename Pred>
+__device__ __forceinline__ void put_keep(int n, Pred kept, uint8_t* __restrict__ keep, uint8_t* __restrict__ uflag) {
+  if (!keep && !uflag) return;
+  for (int j = threadIdx.x; j < n; j += NT) {
+    const bool k = kept(j);
+    if (keep) keep[j] = (uint8_t)(k ? 1 : 0);
+    if (uflag && k) uflag[j] = 1;
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT) k_select_topk(const void* __restrict__ x, int xdt, const float* __restrict__ c,
                                                     int n, int K, int ld, int32_t* __restrict__ idx,
-                                                    float* __restrict__ xs, float* __restrict__ scores) {
+                                                    float* __restrict__ xs, float* __restrict__ scores,
+                                                    uint8_t* __restrict__ keep, uint8_t* __restrict__ uflag) {
   extern __shared__ __align__(16) uint32_t sm[];
   uint32_t* keys = sm;                 // [n]
   uint32_t* hist = sm + n;             // [kSelBins]
@@ -48,6 +61,7 @@ __global__ void __launch_bounds__(NT) k_select_topk(const void* __restrict__ x, 
         idx[ob + pos] = i;
         if (xs) xs[ob + pos] = load_elem(x, xdt, off + i);
       });
+  put_keep<NT>(n, [&](int i) { return kept_by(t, keys[i], i); }, keep ? keep + off : nullptr, uflag);
 }
 
 // The same gate for vectors of up to 16384 channels: one CTA of 1024 threads per token with
@@ -57,7 +71,8 @@ template <int KMAX>
 __global__ void __launch_bounds__(kDT, 1) k_select_topk_regs(const void* __restrict__ x, int xdt,
                                                              const float* __restrict__ c, int n, int K, int ld,
                                                              int32_t* __restrict__ idx, float* __restrict__ xs,
-                                                             float* __restrict__ scores) {
+                                                             float* __restrict__ scores, uint8_t* __restrict__ keep,
+                                                             uint8_t* __restrict__ uflag) {
   __shared__ uint32_t hist[kSelBins + 256];
   __shared__ uint32_t flags[kDMaxN / 32];
   __shared__ uint32_t red[kDW + 1];
@@ -91,13 +106,16 @@ __global__ void __launch_bounds__(kDT, 1) k_select_topk_regs(const void* __restr
     if (xs) xs[ob + at] = load_elem(x, xdt, off + j);
     ++at;
   }
+  put_keep<kDT>(n, [&](int j) { return ((flags[j >> 5] >> (j & 31)) & 1u) != 0u; }, keep ? keep + off : nullptr,
+                uflag);
 }
 
 template <int NT>
 __global__ void __launch_bounds__(NT) k_stat_threshold(const void* __restrict__ v, int vdt, int n, double z,
                                                        int32_t* __restrict__ idx, float* __restrict__ xs,
                                                        int32_t* __restrict__ count, float* __restrict__ tout, int cap,
-                                                       int32_t* status) {
+                                                       int32_t* status, uint8_t* __restrict__ keep,
+                                                       uint8_t* __restrict__ uflag) {
   extern __shared__ __align__(16) float vals[];  // [n]
   __shared__ double dred[NT / 32];
   __shared__ uint32_t wsm[2 * NT / 32 + 1];
@@ -135,28 +153,30 @@ __global__ void __launch_bounds__(NT) k_stat_threshold(const void* __restrict__ 
     if (tout) tout[b] = (float)t;
     if ((int64_t)total > cap) record_status(status, WINA_ERR_CAPACITY);
   }
+  put_keep<NT>(n, [&](int i) { return (double)vals[i] > t; }, keep ? keep + off : nullptr, uflag);
 }
 
 wina_status_t launch_select_topk(const void* x, int xdt, const float* c, int n, int k, int batch, int32_t* idx,
-                                 float* xs, int ld, float* scores, cudaStream_t s) {
+                                 float* xs, int ld, float* scores, cudaStream_t s, uint8_t* keep, uint8_t* uflag) {
   if (n <= kDMaxN) {
     const int kpt = (n + kDT - 1) / kDT;
-    void (*kern)(const void*, int, const float*, int, int, int, int32_t*, float*, float*) =
+    void (*kern)(const void*, int, const float*, int, int, int, int32_t*, float*, float*, uint8_t*, uint8_t*) =
         kpt <= 4 ? k_select_topk_regs<4> : kpt <= 8 ? k_select_topk_regs<8> : kpt <= 12 ? k_select_topk_regs<12>
                                                                                      : k_select_topk_regs<16>;
-    kern<<<batch, kDT, 0, s>>>(x, xdt, c, n, k, ld, idx, xs, scores);
+    kern<<<batch, kDT, 0, s>>>(x, xdt, c, n, k, ld, idx, xs, scores, keep, uflag);
     return cuda_status(cudaGetLastError());
   }
   const size_t smem = (size_t)(n + kSelBins + 2 * kSelCand) * 4;
   return cuda_status(launch_kernel(k_select_topk<kNT>, dim3(batch), dim3(kNT), smem, s, false, x, xdt, c, n, k, ld,
-                                   idx, xs, scores));
+                                   idx, xs, scores, keep, uflag));
 }
 
 wina_status_t launch_stat_threshold(const void* v, int vdt, int n, double z, int batch, int32_t* idx, float* xs,
-                                    int32_t* count, float* t, int cap, int32_t* status_dev, cudaStream_t s) {
+                                    int32_t* count, float* t, int cap, int32_t* status_dev, cudaStream_t s,
+                                    uint8_t* keep, uint8_t* uflag) {
   const size_t smem = (size_t)n * 4;
   return cuda_status(launch_kernel(k_stat_threshold<kNT>, dim3(batch), dim3(kNT), smem, s, false, v, vdt, n, z, idx,
-                                   xs, count, t, cap, status_dev));
+                                   xs, count, t, cap, status_dev, keep, uflag));
 }
 
 }  // namespace wina

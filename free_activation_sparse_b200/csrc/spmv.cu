@@ -133,12 +133,17 @@ __global__ void k_silu_mul(const float* __restrict__ g, const float* __restrict_
 
 static size_t spmv_smem() { return (size_t)kRowChunk * 8 + (size_t)kNT * 8 * 4; }
 
+uint8_t* union_flags_for(void* ws, int wdt, int64_t n, int64_t m, int64_t batch) {
+  if (batch < kUnionMinBatch || batch > kUnionBlock || !union_path_takes(wdt, n, m, batch)) return nullptr;
+  return reinterpret_cast<uint8_t*>((char*)ws + spmv_ws_layout(m, batch).total + union_ws_layout(n, batch).flag);
+}
+
 wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx,
                                    const float* xs, int k, const int32_t* count, int ld_idx, int batch, float* y,
-                                   void* ws, int32_t* status_dev, cudaStream_t s) {
+                                   void* ws, int32_t* status_dev, cudaStream_t s, bool premarked) {
   if (batch >= kUnionMinBatch && union_path_takes(wdt, n, m, batch))
     return launch_union_matvec(Wt, n, m, idx, xs, k, count, ld_idx, batch, y,
-                               (char*)ws + spmv_ws_layout(m, batch).total, status_dev, s);
+                               (char*)ws + spmv_ws_layout(m, batch).total, status_dev, s, premarked);
   if (batch == 1) {  // one token: the single-token kernel's row stream, when it takes the shape
     const SpmvWs L1 = spmv_ws_layout(m, 1);
     const wina_status_t r1 = launch_spmv_one(Wt, wdt, n, m, idx, xs, k, count, ld_idx, y,

@@ -30,7 +30,7 @@
 namespace wina {
 
 constexpr int kUT = 192;           // threads: warp 0 loads, warp 1 issues MMAs, warps 2-5 drain D
-constexpr int kUBlock = 256;       // tokens per block (the MMA's largest N)
+constexpr int kUBlock = kUnionBlock;  // tokens per block (the MMA's largest N)
 constexpr int kUChunk = 64;        // union rows per pipeline stage (one 128-byte swizzle span of X~)
 constexpr int kUMaxStages = 8;
 constexpr int kDenseMin = 20;      // members of a 64-channel block that make it a tile chunk
@@ -56,17 +56,21 @@ __global__ void k_union_mark(const int32_t* __restrict__ idx, int ld, int k, con
   }
 }
 
-// Chunk plan of the union (one CTA of 1024 threads, n <= 65536): thread q counts the
-// members of channel block [64q, 64q + 64); blocks with at least kDenseMin members become
-// tile chunks (in block order), the members of the others are packed into gather chunks
-// after them. Per block: base[q] = the X~ column of its first slot. chunk_row[c] = the first
-// channel of tile chunk c, -1 for a gather chunk. info[0] = chunks, info[1] = 1 (bf16 parts
-// of X~, raised later), info[2] = tile chunks. The padding slots of the last gather chunk
-// point at channel 0 (their inputs are zero).
-__global__ void __launch_bounds__(1024) k_union_plan(const uint8_t* __restrict__ flag, int n, int32_t* __restrict__ base,
-                                                     int32_t* __restrict__ chunk_row, int32_t* __restrict__ slot,
+// Chunk plan of the union and each member's place (one CTA of 1024 threads, n <= 65536).
+// Thread q counts the members of channel block [64q, 64q + 64); blocks with at least
+// kDenseMin members become tile chunks (in block order), the members of the others are
+// packed into gather chunks after them. chunk_row[c] = the first channel of tile chunk c,
+// -1 for a gather chunk; info[0] = chunks, info[1] = 1 (bf16 parts of X~, raised later),
+// info[2] = tile chunks. Then, block by block (a warp per block), each member's X~ column
+// pos[j] (its slot in a tile chunk, or its packed place in a gather chunk, whose slot then
+// names it) is written and the flags are cleared for the next call. The padding slots of
+// the last gather chunk point at channel 0 (their inputs are zero).
+__global__ void __launch_bounds__(1024) k_union_plan(uint8_t* __restrict__ flag, int n, int32_t* __restrict__ chunk_row,
+                                                     int32_t* __restrict__ slot, int32_t* __restrict__ pos,
                                                      uint32_t* __restrict__ info) {
   __shared__ uint32_t red[33];
+  __shared__ int32_t s_base[1024];
+  __shared__ uint8_t s_dense[1024];
   const int q = threadIdx.x;
   const int nblk = (n + 63) / 64;
   uint32_t cnt = 0;
@@ -88,7 +92,8 @@ __global__ void __launch_bounds__(1024) k_union_plan(const uint8_t* __restrict__
   const uint32_t di = block_excl_scan<1024>(dense ? 1u : 0u, red, &ndense);
   const uint32_t go = block_excl_scan<1024>(dense ? 0u : cnt, red, &ngath);
   if (q < nblk) {
-    base[q] = dense ? (int32_t)(di * 64) : (int32_t)(ndense * 64 + go);
+    s_base[q] = dense ? (int32_t)(di * 64) : (int32_t)(ndense * 64 + go);
+    s_dense[q] = dense ? 1 : 0;
     if (dense) chunk_row[di] = q * 64;
   }
   const uint32_t ngc = (ngath + 63) / 64;
@@ -99,73 +104,89 @@ __global__ void __launch_bounds__(1024) k_union_plan(const uint8_t* __restrict__
     info[1] = 1u;
     info[2] = ndense;
   }
-}
-
-// Each union member's X~ column pos[j] (its slot in a tile chunk, or its packed place in a
-// gather chunk, whose slot then names it); the flags are cleared for the next call.
-// Grid: one CTA of 64 threads per channel block.
-__global__ void __launch_bounds__(64) k_union_scatter(uint8_t* __restrict__ flag, int n, const int32_t* __restrict__ base,
-                                                      const int32_t* __restrict__ chunk_row, const uint32_t* info,
-                                                      int32_t* __restrict__ pos, int32_t* __restrict__ slot) {
-  __shared__ uint32_t s_w0;
-  const int q = blockIdx.x, r = threadIdx.x, j = q * 64 + r;
-  const bool f = j < n && flag[j] != 0;
-  if (j < n) flag[j] = 0;
-  const uint32_t bal = __ballot_sync(0xffffffffu, f);
-  if (r == 0) s_w0 = (uint32_t)__popc(bal);
   __syncthreads();
-  if (!f) return;
-  const int32_t b = base[q];
-  // a tile chunk starts at a multiple of 64 below the gather region and holds this block
-  const bool tile = b < (int32_t)(info[2] * 64) && chunk_row[b / 64] == q * 64;
-  if (tile) {
-    pos[j] = b + r;
-  } else {
-    const uint32_t rank = (r >= 32 ? s_w0 : 0u) + (uint32_t)__popc(bal & ((1u << (r & 31)) - 1u));
-    pos[j] = b + (int32_t)rank;
-    slot[b + rank] = j;
+  // members' places, a warp per 64-channel block (lane l: channels 64q + l and 64q + 32 + l)
+  const int warp = q >> 5, lane = q & 31;
+  for (int qb = warp; qb < nblk; qb += 32) {
+    const int j0 = qb * 64 + lane, j1 = j0 + 32;
+    const bool f0 = j0 < n && flag[j0] != 0, f1 = j1 < n && flag[j1] != 0;
+    const uint32_t b0 = __ballot_sync(0xffffffffu, f0), b1 = __ballot_sync(0xffffffffu, f1);
+    if (j0 < n) flag[j0] = 0;
+    if (j1 < n) flag[j1] = 0;
+    const int32_t base = s_base[qb];
+    const uint32_t below = (1u << lane) - 1u;
+    if (s_dense[qb]) {
+      if (f0) pos[j0] = base + lane;
+      if (f1) pos[j1] = base + 32 + lane;
+    } else {
+      if (f0) {
+        const int32_t p = base + (int32_t)__popc(b0 & below);
+        pos[j0] = p;
+        slot[p] = j0;
+      }
+      if (f1) {
+        const int32_t p = base + (int32_t)(__popc(b0) + __popc(b1 & below));
+        pos[j1] = p;
+        slot[p] = j1;
+      }
+    }
   }
 }
 
 // X~ of tokens [b0, b0 + nb) as bf16 rows, part p (hi, mid, lo) of token b in row p * NP + b
-// (row stride kmax); the chunks' columns are written, zeros where a token does not keep
-// the slot's channel; rows nb .. NP-1 of each part are zero. info[1] receives the number of
-// parts the block needs (1 when every value is exactly a bf16).
-__global__ void k_union_xt(const int32_t* __restrict__ idx, const float* __restrict__ xs, int ld, int k,
-                           const int32_t* __restrict__ count, int n, int b0, int nb, int NP,
-                           const int32_t* __restrict__ pos, uint32_t* __restrict__ info, uint16_t* __restrict__ xt,
-                           int kmax) {
+// (row stride kmax): each kept channel's value at its column pos[j]. Every other entry of
+// X~ is zero: the workspace starts zeroed and k_union_clear puts zeros back where this
+// kernel wrote once the product has read them. info[1] receives the number of parts the
+// block needs (1 when every value is exactly a bf16). Grid: (tokens, slices of 256 kept
+// entries).
+__global__ void __launch_bounds__(256) k_union_xt(const int32_t* __restrict__ idx, const float* __restrict__ xs,
+                                                  int ld, int k, const int32_t* __restrict__ count, int n, int b0,
+                                                  int NP, const int32_t* __restrict__ pos, uint32_t* __restrict__ info,
+                                                  uint16_t* __restrict__ xt, int kmax) {
   const int rb = blockIdx.x;
-  const int padded = (int)info[0] * kUChunk;  // X~ columns: 64 per chunk
-  uint16_t* part[3];
-#pragma unroll
-  for (int p = 0; p < 3; ++p) part[p] = xt + ((size_t)p * NP + rb) * kmax;
-  for (int i = threadIdx.x * 8; i < padded; i += blockDim.x * 8)
-#pragma unroll
-    for (int p = 0; p < 3; ++p) *reinterpret_cast<uint4*>(part[p] + i) = make_uint4(0u, 0u, 0u, 0u);
-  if (rb >= nb) return;
-  __syncthreads();
   const int b = b0 + rb;
   const int kb = k >= 0 ? k : max(0, min(__ldg(count + b), ld));
   uint32_t need = 1u;
-  for (int r = threadIdx.x; r < kb; r += blockDim.x) {
+  const int r = blockIdx.y * 256 + threadIdx.x;
+  if (r < kb) {
     const int j = __ldg(idx + (int64_t)b * ld + r);
-    if (j < 0 || j >= n) continue;  // reported by k_union_mark
-    const float v = __ldg(xs + (int64_t)b * ld + r);
-    // v = hi + mid + lo + (a residue below float32 resolution); each difference is exact
-    const uint16_t h = bf16_rn_bits(v);
-    const float r1 = v - __uint_as_float((uint32_t)h << 16);
-    const uint16_t md = bf16_rn_bits(r1);
-    const float r2 = r1 - __uint_as_float((uint32_t)md << 16);
-    const uint16_t l = bf16_rn_bits(r2);
-    const int p = pos[j];
-    part[0][p] = h;
-    part[1][p] = md;
-    part[2][p] = l;
-    need = max(need, (l & 0x7FFFu) ? 3u : ((md & 0x7FFFu) ? 2u : 1u));
+    if (j >= 0 && j < n) {  // out-of-range entries are reported by the marking
+      const float v = __ldg(xs + (int64_t)b * ld + r);
+      // v = hi + mid + lo + (a residue below float32 resolution); each difference is exact
+      const uint16_t h = bf16_rn_bits(v);
+      const float r1 = v - __uint_as_float((uint32_t)h << 16);
+      const uint16_t md = bf16_rn_bits(r1);
+      const float r2 = r1 - __uint_as_float((uint32_t)md << 16);
+      const uint16_t l = bf16_rn_bits(r2);
+      const int p = pos[j];
+      xt[(size_t)rb * kmax + p] = h;
+      xt[((size_t)NP + rb) * kmax + p] = md;
+      xt[((size_t)2 * NP + rb) * kmax + p] = l;
+      need = (l & 0x7FFFu) ? 3u : ((md & 0x7FFFu) ? 2u : 1u);
+    }
   }
   need = __reduce_max_sync(0xffffffffu, need);
   if ((threadIdx.x & 31) == 0 && need > 1u) atomicMax(info + 1, need);
+}
+
+// Zeros back into the entries of X~ that k_union_xt wrote (same grid), after the product.
+__global__ void __launch_bounds__(256) k_union_clear(const int32_t* __restrict__ idx, int ld, int k,
+                                                     const int32_t* __restrict__ count, int n, int b0, int NP,
+                                                     const int32_t* __restrict__ pos, uint16_t* __restrict__ xt,
+                                                     int kmax) {
+  const int rb = blockIdx.x;
+  const int b = b0 + rb;
+  const int kb = k >= 0 ? k : max(0, min(__ldg(count + b), ld));
+  const int r = blockIdx.y * 256 + threadIdx.x;
+  if (r < kb) {
+    const int j = __ldg(idx + (int64_t)b * ld + r);
+    if (j >= 0 && j < n) {
+      const int p = pos[j];
+      xt[(size_t)rb * kmax + p] = 0;
+      xt[((size_t)NP + rb) * kmax + p] = 0;
+      xt[((size_t)2 * NP + rb) * kmax + p] = 0;
+    }
+  }
 }
 
 // Y[b0 + b][m0 .. m0 + 127] += D for this CTA's chunks of U. Grid: (m tiles) x (K splits).
@@ -370,7 +391,6 @@ UnionWs union_ws_layout(int64_t n, int64_t batch) {
   const int64_t nb = batch < kUBlock ? batch : kUBlock;
   w.np = (nb + 15) / 16 * 16;
   w.flag = take((size_t)n);
-  w.base = take((size_t)nblk * 4);
   w.chunk_row = take((size_t)(nblk + 1) * 4);
   w.slot = take((size_t)w.kmax * 4);
   w.pos = take((size_t)n * 4);
@@ -386,11 +406,10 @@ bool union_path_takes(int wdt, int64_t n, int64_t m, int64_t batch) {
 
 wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const int32_t* idx, const float* xs, int k,
                                   const int32_t* count, int ld, int batch, float* y, void* ws, int32_t* status,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, bool premarked) {
   const UnionWs L = union_ws_layout(n, batch);
   char* w = (char*)ws;
   uint8_t* flag = reinterpret_cast<uint8_t*>(w + L.flag);
-  int32_t* base = reinterpret_cast<int32_t*>(w + L.base);
   int32_t* chunk_row = reinterpret_cast<int32_t*>(w + L.chunk_row);
   int32_t* slot = reinterpret_cast<int32_t*>(w + L.slot);
   int32_t* pos = reinterpret_cast<int32_t*>(w + L.pos);
@@ -402,17 +421,19 @@ wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const in
   if (!encode_bf16_2d(&tmX, xt, (uint64_t)L.kmax, (uint64_t)3 * L.np, 64, (uint32_t)L.np)) return WINA_ERR_CUDA;
   const int sms = device_sm_count();
   const int mtiles = (int)((m + 127) / 128);
-  const int nblk = (int)((n + kUChunk - 1) / kUChunk);
   for (int b0 = 0; b0 < batch; b0 += kUBlock) {
     const int nb = std::min(kUBlock, batch - b0);
     const int NP = (nb + 15) / 16 * 16;
     if (NP != L.np) {  // the last, shorter block: its own box height
       if (!encode_bf16_2d(&tmX, xt, (uint64_t)L.kmax, (uint64_t)3 * NP, 64, (uint32_t)NP)) return WINA_ERR_CUDA;
     }
-    k_union_mark<<<nb, 256, 0, s>>>(idx, ld, k, count, (int)n, b0, flag, status);
-    k_union_plan<<<1, 1024, 0, s>>>(flag, (int)n, base, chunk_row, slot, info);
-    k_union_scatter<<<nblk, 64, 0, s>>>(flag, (int)n, base, chunk_row, info, pos, slot);
-    k_union_xt<<<NP, 256, 0, s>>>(idx, xs, ld, k, count, (int)n, b0, nb, NP, pos, info, xt, (int)L.kmax);
+    // the union's flags: marked here from the lists, or already by the gate that made
+    // them (one token block only)
+    if (!(premarked && b0 == 0 && nb == batch)) k_union_mark<<<nb, 256, 0, s>>>(idx, ld, k, count, (int)n, b0, flag, status);
+    k_union_plan<<<1, 1024, 0, s>>>(flag, (int)n, chunk_row, slot, pos, info);
+    const int kcap = k >= 0 ? k : ld;
+    const dim3 xgrid((unsigned)nb, (unsigned)std::max(1, (kcap + 255) / 256));
+    k_union_xt<<<xgrid, 256, 0, s>>>(idx, xs, ld, k, count, (int)n, b0, NP, pos, info, xt, (int)L.kmax);
     cudaError_t e = cudaMemsetAsync(y + (int64_t)b0 * m, 0, (size_t)nb * m * 4, s);
     if (e != cudaSuccess) return cuda_status(e);
     // pipeline depth: up to 8 stages; small token blocks keep the CTA under half an SM's
@@ -429,6 +450,7 @@ wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const in
     if (e != cudaSuccess) return cuda_status(e);
     k_union_gemm<<<mtiles * ksplit, kUT, smem, s>>>(tmA, tmT, tmX, chunk_row, slot, info, (int)m, nb, NP, ksplit, y,
                                                     b0, (int)smem, status);
+    k_union_clear<<<xgrid, 256, 0, s>>>(idx, ld, k, count, (int)n, b0, NP, pos, xt, (int)L.kmax);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e);
   }
