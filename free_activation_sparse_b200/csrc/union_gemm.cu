@@ -137,14 +137,21 @@ __global__ void __launch_bounds__(1024) k_union_plan(uint8_t* __restrict__ flag,
 // (row stride kmax): each kept channel's value at its column pos[j]. Every other entry of
 // X~ is zero: the workspace starts zeroed and k_union_clear puts zeros back where this
 // kernel wrote once the product has read them. info[1] receives the number of parts the
-// block needs (1 when every value is exactly a bf16). Grid: (tokens, slices of 256 kept
+// block needs (1 when every value is exactly a bf16). The tokens' rows of Y (m floats
+// each, m % 4 == 0) are zeroed for the product's sums. Grid: (tokens, slices of 256 kept
 // entries).
 __global__ void __launch_bounds__(256) k_union_xt(const int32_t* __restrict__ idx, const float* __restrict__ xs,
                                                   int ld, int k, const int32_t* __restrict__ count, int n, int b0,
                                                   int NP, const int32_t* __restrict__ pos, uint32_t* __restrict__ info,
-                                                  uint16_t* __restrict__ xt, int kmax) {
+                                                  uint16_t* __restrict__ xt, int kmax, float* __restrict__ y, int m) {
   const int rb = blockIdx.x;
   const int b = b0 + rb;
+  {  // this CTA's slice of token b's row of Y
+    const int m4 = m / 4;
+    const int q0 = (int)((int64_t)m4 * blockIdx.y / gridDim.y), q1 = (int)((int64_t)m4 * (blockIdx.y + 1) / gridDim.y);
+    float4* yr = reinterpret_cast<float4*>(y + (int64_t)b * m);
+    for (int q = q0 + threadIdx.x; q < q1; q += 256) yr[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const int kb = k >= 0 ? k : max(0, min(__ldg(count + b), ld));
   uint32_t need = 1u;
   const int r = blockIdx.y * 256 + threadIdx.x;
@@ -433,9 +440,8 @@ wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const in
     k_union_plan<<<1, 1024, 0, s>>>(flag, (int)n, chunk_row, slot, pos, info);
     const int kcap = k >= 0 ? k : ld;
     const dim3 xgrid((unsigned)nb, (unsigned)std::max(1, (kcap + 255) / 256));
-    k_union_xt<<<xgrid, 256, 0, s>>>(idx, xs, ld, k, count, (int)n, b0, NP, pos, info, xt, (int)L.kmax);
-    cudaError_t e = cudaMemsetAsync(y + (int64_t)b0 * m, 0, (size_t)nb * m * 4, s);
-    if (e != cudaSuccess) return cuda_status(e);
+    k_union_xt<<<xgrid, 256, 0, s>>>(idx, xs, ld, k, count, (int)n, b0, NP, pos, info, xt, (int)L.kmax, y, (int)m);
+    cudaError_t e;
     // pipeline depth: up to 8 stages; small token blocks keep the CTA under half an SM's
     // shared memory so that two CTAs share an SM
     const size_t stage_max = (size_t)2 * kUChunk * 128 + (size_t)3 * NP * 128;
