@@ -515,8 +515,8 @@ def profile_case(name: str) -> None:
     if name == "ffn_decode":
         # the single-token kernel's phase stamps (CTA 0's clock at each phase boundary, read
         # back from the workspace) over 20 more calls, median microseconds per phase
-        phases = ["A keys", "A select", "A flags+list", "B loop", "B store", "barrier 1", "C1 sum",
-                  "barrier 2", "C2 keys", "C2 select", "C2 flags+list", "E loop", "E store", "barrier 3", "E2 sum"]
+        phases = ["A keys", "A select", "A flags+list", "B loop", "B store", "B group sum", "B tail",
+                  "barrier", "C2 keys", "C2 select", "C2 flags+list", "E loop", "E store", "E arrive", "E group sum"]
         mhz = 1965.0  # SM clock under load in the bench's clock samples (the B200's maximum)
         flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
         runs = []

@@ -83,15 +83,17 @@ int max_coresident_grid(K kern, int threads, size_t smem) {
 // workspace layouts
 // ----------------------------------------------------------------------------------
 
-// sparse_matvec: [GridBarrier][partials: kGridCap x (m + 4) float32]. The partial rows
-// are only needed when a token is split over several CTAs (batch < kGridCap).
+// sparse_matvec: [GridBarrier][group counters: kGridCap u32][partials: kGridCap x (m + 4)
+// float32]. The partial rows are only needed when a token is split over several CTAs
+// (batch < kGridCap); the counters serve the single-token column-slice path.
 struct SpmvWs {
-  size_t bar, partials, total;
+  size_t bar, counters, partials, total;
 };
 inline SpmvWs spmv_ws_layout(int64_t m, int64_t batch) {
   SpmvWs w;
   w.bar = 0;
-  w.partials = kAlign;
+  w.counters = kAlign;
+  w.partials = round_up(w.counters + (size_t)kGridCap * 4, kAlign);
   const size_t part = batch < kGridCap ? (size_t)kGridCap * (size_t)(m + 4) * 4 : 0;
   w.total = round_up(w.partials + part, kAlign);
   return w;
@@ -120,13 +122,13 @@ inline size_t spmv_total_ws(int64_t n, int64_t m, int64_t batch) {
 }
 
 // sparse_ffn_swiglu (d, ffn, batch):
-//   bar | h [B][ffn] | keep_g [B][d] | keep_u [B][d] | keep_d [B][ffn] (bytes)
+//   bar | groups [2 * kGridCap] | h [B][ffn] | keep_g [B][d] | keep_u [B][d] | keep_d [B][ffn] (bytes)
 //   | stamps [kFfnStamps] | cta_t [kGridCap][4]
 //   | part [2 * kGridCap][pstride] | dkeys [ffn]        (one token: the single-token kernel)
 //   | idx_gate, idx_up [B][d] | idx_down [B][ffn] | cnt [3][B] | xs_gate, xs_up [B][d]
 //   | xs_down [B][ffn] | g, u [B][ffn] | spmv ws         (the batched path)
 struct FfnWs {
-  size_t bar, h, keep_g, keep_u, keep_d, stamps, cta_t, part, pstride, dkeys, idx_gate, idx_up, idx_down, cnt,
+  size_t bar, groups, h, keep_g, keep_u, keep_d, stamps, cta_t, part, pstride, dkeys, idx_gate, idx_up, idx_down, cnt,
       xs_gate, xs_up, xs_down, g, u, spmv, total;
 };
 inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
@@ -139,6 +141,8 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   };
   const bool one = B == 1;
   w.bar = take(sizeof(GridBarrier));
+  // arrival counters of the single-token kernel's column groups (zero between calls)
+  w.groups = take((size_t)2 * kGridCap * 4);
   w.h = take((size_t)B * ffn * 4);
   w.keep_g = take((size_t)B * d);
   w.keep_u = take((size_t)B * d);
@@ -195,13 +199,6 @@ size_t dense_ws_size(int64_t d, int64_t ffn);
 wina_status_t launch_union_matvec(const void* Wt, int64_t n, int64_t m, const int32_t* idx, const float* xs, int k,
                                   const int32_t* count, int ld, int batch, float* y, void* ws, int32_t* status,
                                   cudaStream_t s, bool premarked = false);
-// One token's sparse product on the single-token FFN kernel's row stream (ffn_decode.cu):
-// part has room for 2 * min(SMs, kGridCap / 2) rows of m + 4 floats; bar is a grid
-// barrier of the workspace. Returns WINA_ERR_UNSUPPORTED_DTYPE without launching when the
-// shape is outside what it takes.
-wina_status_t launch_spmv_one(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx, const float* xs,
-                              int k, const int32_t* count, int ld, float* y, float* part, GridBarrier* bar,
-                              int32_t* status, cudaStream_t st);
 // The single-token FFN kernel (ffn_decode.cu). Returns WINA_ERR_UNSUPPORTED_DTYPE without
 // launching anything when the shape is outside what it takes.
 wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int mode, int k_gate, int k_up,

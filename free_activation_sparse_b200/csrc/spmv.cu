@@ -8,7 +8,15 @@
 // registers and writes one partial row. When P > 1 the launch is cooperative: after a
 // grid barrier (bounded wait) every CTA sums a slice of the outputs over the P partials
 // in a fixed order, so results are bit-reproducible. When P == 1 the CTA writes y.
+//
+// One token: a grid of CG column groups x RG row groups (colstream.cuh). CTA (cg, rg)
+// streams the column slice of group cg of every kept row of rank = rg (mod RG), and the
+// last CTA of a column group to finish sums the group's RG partial rows in order; no
+// grid barrier, and the result is bit-reproducible.
 
+#include <algorithm>
+
+#include "colstream.cuh"
 #include "internal.h"
 
 namespace wina {
@@ -138,17 +146,105 @@ uint8_t* union_flags_for(void* ws, int wdt, int64_t n, int64_t m, int64_t batch)
   return reinterpret_cast<uint8_t*>((char*)ws + spmv_ws_layout(m, batch).total + union_ws_layout(n, batch).flag);
 }
 
+// One token, column slices: CTA b = (cg = b % CG, rg = b / CG). Dynamic SMEM: the CTA's list
+// entries (rows, values) [cap] each, then kCT * 4 floats for the pass sums.
+template <bool BF16, int U>
+__global__ void __launch_bounds__(kCT, 1)
+    k_spmv_cols(const void* __restrict__ Wt, int64_t n, int64_t V, const int32_t* __restrict__ idx,
+                const float* __restrict__ xs, int k_fixed, const int32_t* __restrict__ count, int ld, int CG, int RG,
+                int cap, float* __restrict__ y, float* __restrict__ part, int pstride, unsigned* counters,
+                int32_t* status) {
+  constexpr int EPV = VecOps<BF16>::EPV;
+  extern __shared__ __align__(16) unsigned char smraw[];
+  int32_t* lrow = reinterpret_cast<int32_t*>(smraw);
+  float* lval = reinterpret_cast<float*>(lrow + cap);
+  float* red = lval + cap;  // 16-byte aligned: cap % 4 == 0
+  const int t = threadIdx.x;
+  const int cg = blockIdx.x % CG, rg = blockIdx.x / CG;
+  const int v0 = (int)(V * cg / CG), v1 = (int)(V * (cg + 1) / CG), nv = v1 - v0;
+  int kb = k_fixed;
+  if (kb < 0) kb = max(0, min(__ldg(count), ld));
+  const int cnt = kb > rg ? min(cap, (kb - rg + RG - 1) / RG) : 0;  // cap holds every entry (launcher)
+  for (int i = t; i < cnt; i += kCT) {
+    const int e = rg + i * RG;
+    int32_t row = __ldg(idx + e);
+    float v = __ldg(xs + e);
+    if (row < 0 || (int64_t)row >= n) {  // never read outside Wt
+      record_status(status, WINA_ERR_INVALID_ARG);
+      row = 0;
+      v = 0.f;
+    }
+    lrow[i] = row;
+    lval[i] = v;
+  }
+  __syncthreads();
+  float out[EPV];
+  stream_cols<BF16, U>(Wt, V, v0, nv, cnt, [&](int i) { return lrow[i]; }, [&](int i) { return lval[i]; }, red,
+                       l2_evict_first_policy(), out);
+  if (t < nv) {
+    float4* o = reinterpret_cast<float4*>(part + (int64_t)rg * pstride + (int64_t)(v0 + t) * EPV);
+#pragma unroll
+    for (int q = 0; q < EPV / 4; ++q) __stcg(o + q, make_float4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]));
+  }
+  if (!group_arrive_last(counters + cg, RG)) return;
+  // the last of the group: y over its columns = the RG partial rows summed in order
+  if (t < nv) {
+    float s[EPV];
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) s[e] = 0.f;
+    for (int r = 0; r < RG; ++r) {
+      const float4* o = reinterpret_cast<const float4*>(part + (int64_t)r * pstride + (int64_t)(v0 + t) * EPV);
+#pragma unroll
+      for (int q = 0; q < EPV / 4; ++q) {
+        const float4 v = __ldcg(o + q);
+        s[4 * q] += v.x; s[4 * q + 1] += v.y; s[4 * q + 2] += v.z; s[4 * q + 3] += v.w;
+      }
+    }
+    float4* yo = reinterpret_cast<float4*>(y + (int64_t)(v0 + t) * EPV);
+#pragma unroll
+    for (int q = 0; q < EPV / 4; ++q) yo[q] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+  }
+}
+
+// The single-token column-slice launch; WINA_ERR_UNSUPPORTED_DTYPE (no launch) when the
+// shape is outside what it takes.
+static wina_status_t launch_spmv_cols(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx,
+                                      const float* xs, int k, const int32_t* count, int ld, float* y, void* ws,
+                                      int32_t* status, cudaStream_t s) {
+  const bool bf16 = wdt == WINA_BF16;
+  const int64_t V = m * (bf16 ? 2 : 4) / 16;
+  const int sms = device_sm_count();
+  if (sms < 1) return WINA_ERR_CUDA;
+  // CG column groups of RG row groups, about one CTA per SM: slices of about 32 vectors
+  // (512 bytes, long enough for full-rate streaming) with at least four row groups
+  const int CG = (int)std::max<int64_t>(1, std::min<int64_t>(sms / 4, V / 32));
+  const int RG = std::max(1, std::min(16, sms / CG));
+  if ((V + CG - 1) / CG > kCT || CG > kGridCap || RG > 16) return WINA_ERR_UNSUPPORTED_DTYPE;
+  const int kmax = k >= 0 ? k : ld;
+  const int cap = std::max(4, ((kmax + RG - 1) / RG + 3) / 4 * 4);
+  const size_t smem = (size_t)cap * 8 + (size_t)kCT * 4 * 4;
+  if (smem > 200 * 1024) return WINA_ERR_UNSUPPORTED_DTYPE;
+  const SpmvWs L = spmv_ws_layout(m, 1);
+  float* part = reinterpret_cast<float*>((char*)ws + L.partials);
+  unsigned* counters = reinterpret_cast<unsigned*>((char*)ws + L.counters);
+  const int pstride = (int)(m + 4);  // rows offset by 4 floats: one column of successive rows spreads over L2 slices
+  void (*kern)(const void*, int64_t, int64_t, const int32_t*, const float*, int, const int32_t*, int, int, int, int,
+               float*, float*, int, unsigned*, int32_t*) = bf16 ? k_spmv_cols<true, 4> : k_spmv_cols<false, 4>;
+  cudaError_t e = ensure_prefer_l1((const void*)kern);  // the loads in flight live in L1
+  if (e != cudaSuccess) return cuda_status(e);
+  e = launch_kernel(kern, dim3((unsigned)(CG * RG)), dim3(kCT), smem, s, false, Wt, n, V, idx, xs, k, count, ld, CG,
+                    RG, cap, y, part, pstride, counters, status);
+  return cuda_status(e);
+}
+
 wina_status_t launch_sparse_matvec(const void* Wt, int wdt, int64_t n, int64_t m, const int32_t* idx,
                                    const float* xs, int k, const int32_t* count, int ld_idx, int batch, float* y,
                                    void* ws, int32_t* status_dev, cudaStream_t s, bool premarked) {
   if (batch >= kUnionMinBatch && union_path_takes(wdt, n, m, batch))
     return launch_union_matvec(Wt, n, m, idx, xs, k, count, ld_idx, batch, y,
                                (char*)ws + spmv_ws_layout(m, batch).total, status_dev, s, premarked);
-  if (batch == 1) {  // one token: the single-token kernel's row stream, when it takes the shape
-    const SpmvWs L1 = spmv_ws_layout(m, 1);
-    const wina_status_t r1 = launch_spmv_one(Wt, wdt, n, m, idx, xs, k, count, ld_idx, y,
-                                             reinterpret_cast<float*>((char*)ws + L1.partials),
-                                             reinterpret_cast<GridBarrier*>((char*)ws + L1.bar), status_dev, s);
+  if (batch == 1) {  // one token: column slices, when the shape fits
+    const wina_status_t r1 = launch_spmv_cols(Wt, wdt, n, m, idx, xs, k, count, ld_idx, y, ws, status_dev, s);
     if (r1 != WINA_ERR_UNSUPPORTED_DTYPE) return r1;
   }
   const bool bf16 = wdt == WINA_BF16;
