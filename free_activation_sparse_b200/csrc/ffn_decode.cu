@@ -273,9 +273,13 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
       for (int q = 0; q < EPV / 4; ++q) __stcg(o + q, make_float4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]));
     }
     dstamp(a.stamps, 5);
+    // h and the down scores of the slice, if this CTA is its group's last: float4 columns
+    // [q0, q0 + nq); the first down-gate norms are read before the arrival
+    const int q0 = v0 * EPV / 4, nq = nv * EPV / 4;
+    float4 c4t = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < nq && a.mode == WINA_GATE_TOPK) c4t = __ldg(reinterpret_cast<const float4*>(a.c_down) + q0 + t);
+    touch_pages_d(a.wt_down, (size_t)d * ffn * ESZ);
     if (group_arrive_last(a.groups + cgb, rgs)) {
-      // h and the down scores of the slice: float4 columns [v0 EPV / 4, (v0 + nv) EPV / 4)
-      const int q0 = v0 * EPV / 4, nq = nv * EPV / 4;
       for (int i = t; i < nq; i += kDT) {
         const int q = q0 + i;
         float4 g4 = make_float4(0.f, 0.f, 0.f, 0.f), u4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
                                       silu_d(g4.w) * u4.w);
         __stcg(reinterpret_cast<float4*>(a.h) + q, h4);
         if (a.mode == WINA_GATE_TOPK) {
-          const float4 c4 = __ldg(reinterpret_cast<const float4*>(a.c_down) + q);
+          const float4 c4 = i == t ? c4t : __ldg(reinterpret_cast<const float4*>(a.c_down) + q);
           __stcg(reinterpret_cast<uint4*>(a.dkeys) + q,
                  make_uint4(__float_as_uint(fabsf(h4.x * c4.x)), __float_as_uint(fabsf(h4.y * c4.y)),
                             __float_as_uint(fabsf(h4.z * c4.z)), __float_as_uint(fabsf(h4.w * c4.w))));
@@ -300,7 +304,6 @@ __global__ void __launch_bounds__(kDT, 1) k_ffn_decode(DecodeParams a) {
     }
   }
   dstamp(a.stamps, 6);
-  touch_pages_d(a.wt_down, (size_t)d * ffn * ESZ);
   clear_hist(hist);  // for the down selection (red overlays it)
   dstamp(a.stamps, 7);
   if (!grid_sync_fixed(a.bar, G, a.status, a.wait_ns)) return;
@@ -398,13 +401,15 @@ wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int
   if (G < 8) return WINA_ERR_UNSUPPORTED_DTYPE;
   // phase B: four row groups per column group (slices of 37 vectors of a Llama-7B row),
   // split between gate and up in proportion to their kept rows (two each when unknown)
-  int rgg = 2;
-  if (mode == WINA_GATE_TOPK && k_gate + k_up > 0) rgg = (int)((4 * (int64_t)k_gate + (k_gate + k_up) / 2) / (k_gate + k_up));
-  rgg = std::max(1, std::min(3, rgg));
-  const int rgu = 4 - rgg;
-  const int cgb = G / 4;
-  // phase E: slices of about 32 vectors (512 bytes), with at least four row groups
-  const int cge = std::max(1, std::min(G / 4, d * esz / 16 / 32));
+  const int rgs = 4;  // row groups per column group in phase B
+  int rgg = rgs / 2;
+  if (mode == WINA_GATE_TOPK && k_gate + k_up > 0)
+    rgg = (int)((rgs * (int64_t)k_gate + (k_gate + k_up) / 2) / (k_gate + k_up));
+  rgg = std::max(1, std::min(rgs - 1, rgg));
+  const int rgu = rgs - rgg;
+  const int cgb = G / rgs;
+  // phase E: slices of about 64 vectors (1 KB), with at least four row groups
+  const int cge = std::max(1, std::min(G / 4, d * esz / 16 / 64));
   const int rge = std::min(16, G / cge);
   const int V_b = ffn * esz / 16, V_e = d * esz / 16;
   if ((V_b + cgb - 1) / cgb > kCT || (V_e + cge - 1) / cge > kCT || V_b < cgb || V_e < cge)
