@@ -851,7 +851,7 @@ def main():
 def _kernel_sha() -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("common.cuh", "regsel.cuh", "ffn_decode.cu"):
+    for f in ("common.cuh", "regsel.cuh", "colstream.cuh", "ffn_decode.cu"):
         with open(os.path.join(ROOT, "free_activation_sparse_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

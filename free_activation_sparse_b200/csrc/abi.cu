@@ -36,6 +36,34 @@ SmemEntry g_l1[kCacheSlots];
 int g_nl1 = 0;
 }  // namespace
 
+namespace {
+SideStream g_side[kMaxDev];
+bool g_side_ok[kMaxDev];
+std::mutex g_side_mu;
+}  // namespace
+
+bool side_stream(cudaStream_t main, SideStream* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_side_ok[dev]) {
+    // not while `main` is being captured into a graph: creating a stream then is left out
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(main, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
+    SideStream ss;
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaEventCreateWithFlags(&ss.fork_ev, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join_ev, cudaEventDisableTiming) != cudaSuccess)
+      return false;
+    g_side[dev] = ss;
+    g_side_ok[dev] = true;
+  }
+  *out = g_side[dev];
+  return true;
+}
+
+std::unique_lock<std::mutex> side_stream_lock() { return std::unique_lock<std::mutex>(g_side_mu); }
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;

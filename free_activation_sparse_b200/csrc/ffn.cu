@@ -6,7 +6,8 @@
 // The C-ABI entry point. One token takes the single persistent kernel of ffn_decode.cu;
 // several tokens (or shapes that kernel does not take) run as a sequence of batched
 // calls: per projection its gate (which also writes the kept-set bytes and, for the union
-// path, the union's flags) and its sparse product, with silu(g) * u before the down gate.
+// path, the union's flags) and its sparse product, with silu(g) * u before the down gate;
+// the up projection runs on a side stream beside the gate projection.
 #include <math.h>
 
 #include <algorithm>
@@ -68,48 +69,75 @@ extern "C" wina_status_t sparse_ffn_swiglu(const wina_ffn_t* f, const void* x, w
   float* xd = reinterpret_cast<float*>(w + L.xs_down);
   float* g = reinterpret_cast<float*>(w + L.g);
   float* u = reinterpret_cast<float*>(w + L.u);
-  void* sw = w + L.spmv;
+  void* sw = w + L.spmv;    // gate
+  void* sw2 = w + L.spmv2;  // up
+  void* sw3 = w + L.spmv3;  // down
   const int B = (int)batch;
-  // union flags of each projection's product (set by the gate that makes its lists, when
-  // the union path serves the call); gate and up share the workspace, so each gate runs
-  // right before its own product
-  uint8_t* uf_gu = union_flags_for(sw, f->wdt, d, ffn, B);
-  uint8_t* uf_d = union_flags_for(sw, f->wdt, ffn, d, B);
+  // union flags of each projection's product, set by the gate that makes its lists when
+  // the union path serves the call
+  uint8_t* uf_g = union_flags_for(sw, f->wdt, d, ffn, B);
+  uint8_t* uf_u = union_flags_for(sw2, f->wdt, d, ffn, B);
+  uint8_t* uf_d = union_flags_for(sw3, f->wdt, ffn, d, B);
   wina_status_t r;
+  // The gate and up projections are independent until silu(g) * u: up runs on a side
+  // stream beside gate when one is available (fork after the work enqueued so far, join
+  // before silu).
+  SideStream ss;
+  std::unique_lock<std::mutex> lk = side_stream_lock();
+  const bool par = side_stream(st, &ss);
+  cudaStream_t su = st;
+  if (par) {
+    if ((r = cuda_status(cudaEventRecord(ss.fork_ev, st)))) return r;
+    if ((r = cuda_status(cudaStreamWaitEvent(ss.s, ss.fork_ev, 0)))) return r;
+    su = ss.s;
+  }
+  auto join = [&]() -> wina_status_t {
+    if (!par) return WINA_OK;
+    wina_status_t rj = cuda_status(cudaEventRecord(ss.join_ev, su));
+    if (rj == WINA_OK) rj = cuda_status(cudaStreamWaitEvent(st, ss.join_ev, 0));
+    lk.unlock();
+    return rj;
+  };
   if (mode == WINA_GATE_STAT) {
-    // gate and up threshold the same signed x: one kept set serves both
-    if ((r = launch_stat_threshold(x, xdt, (int)d, z, B, ig, xg, cnt, nullptr, (int)d, status_dev, st, keep_g, uf_gu)))
+    // gate and up threshold the same signed x: one kept set serves both (up reads the
+    // lists once they exist, so it waits for the threshold)
+    if ((r = launch_stat_threshold(x, xdt, (int)d, z, B, ig, xg, cnt, nullptr, (int)d, status_dev, st, keep_g, uf_g)))
       return r;
-    if ((r = cuda_status(cudaMemcpyAsync(keep_u, keep_g, (size_t)B * d, cudaMemcpyDeviceToDevice, st)))) return r;
+    if (par) {
+      if ((r = cuda_status(cudaEventRecord(ss.fork_ev, st)))) return r;
+      if ((r = cuda_status(cudaStreamWaitEvent(su, ss.fork_ev, 0)))) return r;
+    }
+    if ((r = cuda_status(cudaMemcpyAsync(keep_u, keep_g, (size_t)B * d, cudaMemcpyDeviceToDevice, su)))) return r;
+    if ((r = launch_sparse_matvec(f->wt_up, f->wdt, d, ffn, ig, xg, -1, cnt, (int)d, B, u, sw2, status_dev, su)))
+      return r;
     if ((r = launch_sparse_matvec(f->wt_gate, f->wdt, d, ffn, ig, xg, -1, cnt, (int)d, B, g, sw, status_dev, st,
-                                  uf_gu != nullptr)))
+                                  uf_g != nullptr)))
       return r;
-    if ((r = launch_sparse_matvec(f->wt_up, f->wdt, d, ffn, ig, xg, -1, cnt, (int)d, B, u, sw, status_dev, st)))
-      return r;
+    if ((r = join())) return r;
     if ((r = launch_silu_mul(g, u, h, (int64_t)B * ffn, st))) return r;
     if ((r = launch_stat_threshold(h, WINA_F32, (int)ffn, z, B, idn, xd, cnt + 2 * B, nullptr, (int)ffn, status_dev,
                                    st, keep_d, uf_d)))
       return r;
-    return launch_sparse_matvec(f->wt_down, f->wdt, ffn, d, idn, xd, -1, cnt + 2 * B, (int)ffn, B, y, sw, status_dev,
+    return launch_sparse_matvec(f->wt_down, f->wdt, ffn, d, idn, xd, -1, cnt + 2 * B, (int)ffn, B, y, sw3, status_dev,
                                 st, uf_d != nullptr);
   }
   const float* cg = mode == WINA_GATE_TOPK ? f->c_gate : nullptr;
   const float* cu = mode == WINA_GATE_TOPK ? f->c_up : nullptr;
   const float* cd = mode == WINA_GATE_TOPK ? f->c_down : nullptr;
-  if ((r = launch_select_topk(x, xdt, cg, (int)d, (int)k_gate, B, ig, xg, (int)d, nullptr, st, keep_g, uf_gu)))
+  if ((r = launch_select_topk(x, xdt, cu, (int)d, (int)k_up, B, iu, xu, (int)d, nullptr, su, keep_u, uf_u))) return r;
+  if ((r = launch_sparse_matvec(f->wt_up, f->wdt, d, ffn, iu, xu, (int)k_up, nullptr, (int)d, B, u, sw2, status_dev,
+                                su, uf_u != nullptr)))
+    return r;
+  if ((r = launch_select_topk(x, xdt, cg, (int)d, (int)k_gate, B, ig, xg, (int)d, nullptr, st, keep_g, uf_g)))
     return r;
   if ((r = launch_sparse_matvec(f->wt_gate, f->wdt, d, ffn, ig, xg, (int)k_gate, nullptr, (int)d, B, g, sw,
-                                status_dev, st, uf_gu != nullptr)))
+                                status_dev, st, uf_g != nullptr)))
     return r;
-  if ((r = launch_select_topk(x, xdt, cu, (int)d, (int)k_up, B, iu, xu, (int)d, nullptr, st, keep_u, uf_gu)))
-    return r;
-  if ((r = launch_sparse_matvec(f->wt_up, f->wdt, d, ffn, iu, xu, (int)k_up, nullptr, (int)d, B, u, sw, status_dev,
-                                st, uf_gu != nullptr)))
-    return r;
+  if ((r = join())) return r;
   if ((r = launch_silu_mul(g, u, h, (int64_t)B * ffn, st))) return r;
   if ((r = launch_select_topk(h, WINA_F32, cd, (int)ffn, (int)k_down, B, idn, xd, (int)ffn, nullptr, st, keep_d,
                               uf_d)))
     return r;
-  return launch_sparse_matvec(f->wt_down, f->wdt, ffn, d, idn, xd, (int)k_down, nullptr, (int)ffn, B, y, sw,
+  return launch_sparse_matvec(f->wt_down, f->wdt, ffn, d, idn, xd, (int)k_down, nullptr, (int)ffn, B, y, sw3,
                               status_dev, st, uf_d != nullptr);
 }

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "wina.h"
 
@@ -43,6 +45,18 @@ cudaError_t ensure_smem_limit(const void* kern, size_t smem);
 cudaError_t ensure_prefer_l1(const void* kern);
 // Shared-memory carveout preference of a kernel, in percent of the maximum (cached).
 cudaError_t ensure_carveout(const void* kern, int pct);
+
+// A second stream of the current device, with two events, for work that can run beside
+// the caller's stream (created once per device, non-blocking). Returns false when none is
+// available (then everything runs on the caller's stream). `fork` makes the side stream
+// wait for the work enqueued so far on `main`; `join` makes `main` wait for the side
+// stream's work. Host threads enqueueing fork...join pairs are serialised by `lock`.
+struct SideStream {
+  cudaStream_t s;
+  cudaEvent_t fork_ev, join_ev;
+};
+bool side_stream(cudaStream_t main, SideStream* out);
+std::unique_lock<std::mutex> side_stream_lock();
 
 // Co-resident CTAs per SM of `kern` at this block size and SMEM on the current device
 // (cached per device, kernel, block size and SMEM). 0 on error.
@@ -126,10 +140,10 @@ inline size_t spmv_total_ws(int64_t n, int64_t m, int64_t batch) {
 //   | stamps [kFfnStamps] | cta_t [kGridCap][4]
 //   | part [2 * kGridCap][pstride] | dkeys [ffn]        (one token: the single-token kernel)
 //   | idx_gate, idx_up [B][d] | idx_down [B][ffn] | cnt [3][B] | xs_gate, xs_up [B][d]
-//   | xs_down [B][ffn] | g, u [B][ffn] | spmv ws         (the batched path)
+//   | xs_down [B][ffn] | g, u [B][ffn] | spmv ws of gate, up, down   (the batched path)
 struct FfnWs {
   size_t bar, groups, h, keep_g, keep_u, keep_d, stamps, cta_t, part, pstride, dkeys, idx_gate, idx_up, idx_down, cnt,
-      xs_gate, xs_up, xs_down, g, u, spmv, total;
+      xs_gate, xs_up, xs_down, g, u, spmv, spmv2, spmv3, total;
 };
 inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   FfnWs w;
@@ -165,8 +179,11 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   w.xs_down = take((size_t)B * ffn * 4);
   w.g = take((size_t)B * ffn * 4);
   w.u = take((size_t)B * ffn * 4);
-  const int64_t mmax = ffn > d ? ffn : d;
-  w.spmv = take(spmv_total_ws(mmax, mmax, B));
+  // the products' workspaces: gate, up (its own, so that it can run beside the gate's),
+  // down (its own shape: the union path keeps parts of its workspace zero between calls)
+  w.spmv = take(spmv_total_ws(d, ffn, B));
+  w.spmv2 = take(spmv_total_ws(d, ffn, B));
+  w.spmv3 = take(spmv_total_ws(ffn, d, B));
   w.total = o;
   return w;
 }

@@ -214,11 +214,21 @@ wina_status_t stat_topk_threshold(const void* v, wina_dtype_t vdt, int64_t n, do
 
 /* Sparse product over the kept channels ("Spark Transformer", section 3.1, SVMM):
  *   y[b][:] = sum over r < k_b of xs[b][r] * Wt[idx[b][r]][:]      for b < batch,
- * reading only the kept rows of the input-major weight. The co-resident grid is shared
- * among the tokens: token b gets P = grid / batch CTAs (at least one), which split its
- * kept rows (split-K) and, when P > 1, sum their partial rows in a fixed order after a
- * grid barrier, so results are bit-reproducible. Each token reads its own kept rows: a
- * row kept by several tokens is read once per token.
+ * reading only the kept rows of the input-major weight.
+ *   One token: the grid is split into column groups x row groups; a CTA streams its
+ *   column group's slice of every kept row of its row group (rank = row group modulo
+ *   the number of row groups), and the last CTA of a column group adds the group's few
+ *   partial rows in a fixed order. No grid barrier; bit-reproducible.
+ *   Two or three tokens, or f32 weights: the co-resident grid is shared among the
+ *   tokens; token b gets P = grid / batch CTAs (at least one), which split its kept rows
+ *   and, when P > 1, sum their partial rows in a fixed order after a grid barrier
+ *   (bit-reproducible). Each token reads its own kept rows.
+ *   Four or more tokens with bf16 weights: per block of up to 256 tokens, the union U
+ *   of their kept rows is read once, whatever the number of tokens that keep each row,
+ *   and Y = X~ . Wt[U,:] runs on the tcgen05 tensor cores (X~: each token's value at
+ *   each union row or 0, split into bf16 parts that reproduce it to float32 precision);
+ *   the split of U over CTAs adds into y with float atomics, so the last bits of y may
+ *   differ from call to call.
  *   Wt:    device [n][m] of wdt (m % 8 == 0 and m <= 32768 for bf16; m % 4 == 0 and
  *          m <= 16384 for f32).
  *   idx:   device int32 [batch][ld_idx]: kept input channels of each token (any order;
@@ -239,8 +249,9 @@ wina_status_t sparse_matvec(const void* Wt, wina_dtype_t wdt, int64_t n, int64_t
  * such entry point; it exists for code that runs where device allocation is not an
  * option (a framework that owns a fixed device memory pool, a latency-critical loop in
  * which cudaMalloc could synchronise the device, a plugin that is only handed input and
- * output buffers). Same arguments and results as sparse_matvec, minus ws / ws_bytes:
- * the scratch (a barrier word pair and the split-K partial rows) lives in a fixed
+ * output buffers). Same arguments and results as sparse_matvec, minus ws / ws_bytes,
+ * always computed by the split-K product (every token on its own CTAs, no union): the
+ * scratch (a barrier word pair and the split-K partial rows) lives in a fixed
  * 8 MiB + 256 B array of device memory declared by the library, which every GPU that
  * loads the library holds until the process exits. It allocates nothing.
  *   Limit: when batch is smaller than the co-resident grid (148 CTAs on a B200), a
@@ -248,10 +259,10 @@ wina_status_t sparse_matvec(const void* Wt, wina_dtype_t wdt, int64_t n, int64_t
  *   so batch * m <= 1,048,576 is required (at least two partial rows per token);
  *   larger calls return WINA_ERR_INVALID_ARG. With batch at least the grid, each
  *   token has its own CTA, the array is not used and any size is accepted.
- *   The first call on a device looks up the array's device address (once per device,
- *   with that device current) and keeps it for the life of the process; make that
- *   first call before any stream capture, and do not use this entry point on a device
- *   after cudaDeviceReset (the kept address would be stale).
+ *   Every call looks up the array's device address in the current device's context
+ *   (cudaGetSymbolAddress, a cheap query), so the entry point stays valid across
+ *   cudaDeviceReset; the first call on a device may also load the library's device
+ *   code, so make it before any stream capture.
  *   Every call clears the barrier words on `stream` and then reuses the same array:
  *   calls that overlap on the GPU (other streams, other threads) race and must not
  *   be issued. */
@@ -270,17 +281,20 @@ wina_status_t sparse_matvec_noalloc(const void* Wt, wina_dtype_t wdt, int64_t n,
  * projection's signed input (k_* ignored; gate and up then share one kept set); with
  * WINA_GATE_DENSE every channel is kept.
  * One token (d, ffn <= 16384) runs as one persistent cooperative kernel with one CTA of
- * 1024 threads per SM: each SM works on the gate or the up projection, selects that
- * projection's kept channels itself (the keys in registers, a radix select on their
- * bits), takes every (number of SMs on that projection)-th kept row in ascending order
- * and streams those rows with 16-byte loads into a partial row of g or u; after a grid
- * barrier each SM sums its slice of the columns over all partial rows in a fixed order
- * and writes h and the down scores for it; after a second barrier every SM selects the
- * down kept set and streams its share of those rows into a partial row of y, which a
- * third barrier and a last fixed-order slice sum turn into y. Every barrier wait is
- * bounded in time. Kept sets are exact and every sum is taken in a fixed order, so
- * repeated calls give identical bits. Several tokens (or wider shapes) run as a sequence
- * of the batched calls above.
+ * 1024 threads per SM. The SMs form column groups of the ffn outputs, each with four row
+ * groups split between gate and up: every SM selects its projection's kept channels
+ * itself (the keys in registers, a radix select on their bits), takes the kept rows of
+ * its row group (every fourth, or so, in ascending order) and streams its column group's
+ * slice of them with 16-byte loads into a partial row; the last SM of a column group adds
+ * the group's partials in a fixed order and writes h and the down scores for the slice.
+ * After the one grid barrier every SM selects the down kept set and streams its slice of
+ * its row group's down rows the same way; the last SM of each column group adds those
+ * partials into y. The barrier wait is bounded in time. Kept sets are exact and every
+ * sum is taken in a fixed order, so repeated calls give identical bits. Several tokens
+ * (or wider shapes) run as a sequence of the batched calls above, the up projection on a
+ * side stream of the library beside the gate projection (one stream and two events per
+ * device, created on the first such call outside stream capture and joined back to
+ * `stream` by events, so graph capture of `stream` includes them).
  *   f:   host pointer to the weight descriptor (read during the call only).
  *   x:   device [batch][d] of xdt.   y: device float32 [batch][d] (written).
  *   k_gate, k_up in [0, d]; k_down in [0, ffn] (WINA_GATE_TOPK).  0 < s < 1 (STAT).
