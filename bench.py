@@ -732,7 +732,7 @@ def main():
     matvec_bs1 = {
         "gate_4096x11008_k%d" % kg: dict(_frac(kg * FFN * 2 + kg * 8 + FFN * 4, us_mg, peak), us_per_call=us_mg),
         "down_11008x4096_k%d" % kd: dict(_frac(kd * D * 2 + kd * 8 + D * 4, us_md, peak), us_per_call=us_md),
-        "kernel": "k_sparse_matvec (split-K over all SMs, fixed-order partial sums)"}
+        "kernel": "k_spmv_cols (column groups x row groups, the last CTA of a column group sums its partials in order)"}
     del sel_g, sel_d, yg, ydn, mws
 
     # several tokens (the batched path): 16 tokens per call on the same layers; effective

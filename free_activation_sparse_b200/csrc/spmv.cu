@@ -216,10 +216,10 @@ static wina_status_t launch_spmv_cols(const void* Wt, int wdt, int64_t n, int64_
   const int sms = device_sm_count();
   if (sms < 1) return WINA_ERR_CUDA;
   // CG column groups of RG row groups, about one CTA per SM: slices of about 32 vectors
-  // (512 bytes, long enough for full-rate streaming) with at least four row groups
+  // (512 bytes, long enough for full-rate streaming), the rest of the SMs as row groups
   const int CG = (int)std::max<int64_t>(1, std::min<int64_t>(sms / 4, V / 32));
-  const int RG = std::max(1, std::min(16, sms / CG));
-  if ((V + CG - 1) / CG > kCT || CG > kGridCap || RG > 16) return WINA_ERR_UNSUPPORTED_DTYPE;
+  const int RG = std::max(1, std::min(64, sms / CG));
+  if ((V + CG - 1) / CG > kCT || CG > kGridCap || RG > 64) return WINA_ERR_UNSUPPORTED_DTYPE;
   const int kmax = k >= 0 ? k : ld;
   const int cap = std::max(4, ((kmax + RG - 1) / RG + 3) / 4 * 4);
   const size_t smem = (size_t)cap * 8 + (size_t)kCT * 4 * 4;
