@@ -408,7 +408,8 @@ wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int
   rgg = std::max(1, std::min(rgs - 1, rgg));
   const int rgu = rgs - rgg;
   const int cgb = G / rgs;
-  // phase E: slices of about 64 vectors (1 KB), with at least four row groups
+  // phase E: slices of about 64 vectors (1 KB), at most 16 row groups (8 x 16 CTAs for
+  // Llama-7B's d = 4096; 16 x 9 slices of 512 B streamed slower)
   const int cge = std::max(1, std::min(G / 4, d * esz / 16 / 64));
   const int rge = std::min(16, G / cge);
   const int V_b = ffn * esz / 16, V_e = d * esz / 16;
