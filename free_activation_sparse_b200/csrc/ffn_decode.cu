@@ -420,7 +420,7 @@ wina_status_t launch_ffn_decode(const wina_ffn_t* f, const void* x, int xdt, int
   const DecodeSmem SL = decode_smem(nmax, cap);
   const size_t smem = SL.total;
   if (smem > 96 * 1024) return WINA_ERR_UNSUPPORTED_DTYPE;  // keep most of the L1 for the loads in flight
-  if ((size_t)(rgg + rgu + rge) > 2 * (size_t)kGridCap) return WINA_ERR_UNSUPPORTED_DTYPE;
+  if (rgg + rgu + rge > kDecodeRows) return WINA_ERR_UNSUPPORTED_DTYPE;
   {
     cudaError_t e = ensure_smem_limit(kern, smem);  // static shared memory comes on top of the dynamic part
     if (e != cudaSuccess) return cuda_status(e);

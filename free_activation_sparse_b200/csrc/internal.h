@@ -19,6 +19,7 @@ constexpr int kNT = 512;          // threads per CTA of the selection / product 
 constexpr int kRowChunk = 1024;   // kept rows staged in SMEM at a time by sparse_matvec
 constexpr size_t kAlign = 256;    // alignment of every workspace sub-buffer
 constexpr int kFfnStamps = 32;  // phase clock stamps the single-token FFN kernel leaves (16 used)
+constexpr int kDecodeRows = 32;  // partial rows of the single-token FFN kernel (its row groups: at most 4 + 16)
 
 inline bool valid_dtype(int dt) { return dt == WINA_F32 || dt == WINA_BF16; }
 inline int64_t elem_size(int dt) { return dt == WINA_BF16 ? 2 : 4; }
@@ -138,7 +139,7 @@ inline size_t spmv_total_ws(int64_t n, int64_t m, int64_t batch) {
 // sparse_ffn_swiglu (d, ffn, batch):
 //   bar | groups [2 * kGridCap] | h [B][ffn] | keep_g [B][d] | keep_u [B][d] | keep_d [B][ffn] (bytes)
 //   | stamps [kFfnStamps] | cta_t [kGridCap][4]
-//   | part [2 * kGridCap][pstride] | dkeys [ffn]        (one token: the single-token kernel)
+//   | part [kDecodeRows][pstride] | dkeys [ffn]        (one token: the single-token kernel)
 //   | idx_gate, idx_up [B][d] | idx_down [B][ffn] | cnt [3][B] | xs_gate, xs_up [B][d]
 //   | xs_down [B][ffn] | g, u [B][ffn] | spmv ws of gate, up, down   (the batched path)
 struct FfnWs {
@@ -166,7 +167,7 @@ inline FfnWs ffn_ws_layout(int64_t d, int64_t ffn, int64_t B) {
   // partial rows: a multiple of 4 floats plus 4, so that the same column of successive
   // rows (read together when the rows are summed) does not fall on one L2 slice
   w.pstride = (size_t)((ffn > d ? ffn : d) + 3) / 4 * 4 + 4;
-  w.part = take(one ? (size_t)2 * kGridCap * w.pstride * 4 : 0);
+  w.part = take(one ? (size_t)kDecodeRows * w.pstride * 4 : 0);
   w.dkeys = take(one ? (size_t)ffn * 4 : 0);
   // the batched path (several tokens, or one token of a shape the single-token kernel
   // does not take)
